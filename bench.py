@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward TFLOP/s on B200 (causal bf16, B=4 H=16 N=4096 d=128).
+
+One step = one forward (one launch of the attention kernel) over the whole
+workload with inputs resident in HBM.  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload c3] [--no-cpu-baseline]
+
+FLOPs are algorithmic: 4 * d * (kept query-key pairs) per head, summed over
+B * H heads (the causal mask keeps N (N + 1) / 2 pairs); masked work is not
+counted.  Between timed steps the inputs rotate over two sets of device
+buffers whose combined size is several times the 126 MB L2, so no step reads
+its inputs from L2 left warm by the step before.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s & % of B200 BF16 tensor peak (causal, N=4096, d=128)"
+SPEC_BF16_TFLOPS = 2250.0
+L2_BYTES = 126 * 2 ** 20
+KERNEL_SOURCES = ["exact_tiled_attention_44_b200/csrc/attn_kernel.cuh",
+                  "exact_tiled_attention_44_b200/csrc/ptx.cuh",
+                  "exact_tiled_attention_44_b200/csrc/attn_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    if d.get("kernel_src_sha256") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str | None = None):
+        self.path = path or tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.t_begin = self.t_end = None
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu_index)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_begin(self):
+        self.t_begin = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[1].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + parts[1].split(".")[1]) if "." in parts[1] else 0.0
+                rows.append((ts + frac, float(parts[2]), float(parts[3]), float(parts[4]), parts[5:]))
+            except (ValueError, IndexError):
+                continue
+        window = "timed"
+        sel = [r for r in rows if self.t_begin and self.t_begin - 0.05 <= r[0] <= self.t_end + 0.05]
+        if not sel:
+            sel, window = rows, "whole run (timed region shorter than the sampling interval)"
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in sel:
+            for nm, val in zip(names, r[4][1:5]):
+                if val.strip().lower() in ("active", "1", "yes"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": max(r[2] for r in sel),
+                "power_w_max": max(r[3] for r in sel), "samples": len(sel), "window": window,
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- oracle leg
+
+def _oracle_rows_task(args):
+    """Worker: the oracle for query rows [r0, r1) of one head; returns seconds spent."""
+    import numpy as np
+    import oracle
+    Qh, Kh, Vh, scale, causal, window, n_sink, r0, r1 = args
+    t0 = time.perf_counter()
+    oracle.attention_bh(Qh, Kh, Vh, 0, 0, scale, causal, window, n_sink, rows=np.arange(r0, r1))
+    return time.perf_counter() - t0
+
+
+def _head_arrays(w, q, k, v, b, h):
+    from exact_tiled_attention_44_b200.inputs import to_f64
+    g = h // (w.H // w.H_kv)
+    return (to_f64(q[b:b + 1, h:h + 1]), to_f64(k[b:b + 1, g:g + 1]), to_f64(v[b:b + 1, g:g + 1]))
+
+
+def _pairs_rows(w, r0, r1):
+    """Kept pairs of query rows [r0, r1) (mask rule restated for accounting)."""
+    tot = 0
+    for i in range(r0, r1):
+        if not w.causal:
+            tot += w.N
+        elif w.window <= 0 or w.window >= w.N:
+            tot += i + 1
+        else:
+            tot += min(i + 1, w.window) + max(0, min(w.n_sink, i - w.window + 1))
+    return tot
+
+
+def cpu_oracle_throughput(name: str, q, k, v, budget_s: float = 20.0):
+    """The float64 oracle, as it stands, on a bounded sample of the workload.
+
+    Chunks of complete query rows of distinct heads are spread over all host
+    cores (one BLAS thread per worker process, spawn start method; the parent
+    sends each worker only the head it needs).  Returns the cpu_baseline
+    object in TFLOP/s.
+    """
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    from exact_tiled_attention_44_b200.inputs import WORKLOADS
+    w = WORKLOADS[name]
+    cores = len(os.sched_getaffinity(0))
+    rows_per_task = 256
+    saved = {kk: os.environ.get(kk) for kk in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for kk in saved:
+        os.environ[kk] = "1"
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    arrays = {}
+
+    def task(i):
+        b, h = heads[i % len(heads)]
+        if (b, h) not in arrays:
+            arrays[(b, h)] = _head_arrays(w, q, k, v, b, h)
+        n_chunks = (w.N + rows_per_task - 1) // rows_per_task
+        r0 = ((i // len(heads)) * 7 % n_chunks) * rows_per_task
+        return arrays[(b, h)] + (w.scale, w.causal, w.window, w.n_sink, r0, min(w.N, r0 + rows_per_task))
+
+    try:
+        ctx = mp.get_context("spawn")
+        with cf.ProcessPoolExecutor(max_workers=cores, mp_context=ctx) as ex:
+            cal = [task(i) for i in range(min(cores, 4))]
+            per_task = max(1e-3, statistics.median(ex.map(_oracle_rows_task, cal)))
+            n_tasks = max(cores, int(budget_s * cores / per_task))
+            tasks = [task(i) for i in range(n_tasks)]
+            t0 = time.perf_counter()
+            list(ex.map(_oracle_rows_task, tasks, chunksize=max(1, n_tasks // (4 * cores))))
+            wall = time.perf_counter() - t0
+    finally:
+        for kk, val in saved.items():
+            if val is None:
+                os.environ.pop(kk, None)
+            else:
+                os.environ[kk] = val
+    flops = sum(4.0 * w.d * _pairs_rows(w, t[7], t[8]) for t in tasks)
+    return {"value": flops / wall / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(tasks)} chunks of {rows_per_task} complete query rows from the "
+                      f"{w.B * w.H} heads of {name}; float64 full score rows; {wall:.1f} s wall "
+                      f"on {cores} worker processes"}
+
+
+def _blas_threads() -> int:
+    """Threads numpy's BLAS uses in this process (the reference arm's core count)."""
+    for kk in ("OPENBLAS_NUM_THREADS", "OMP_NUM_THREADS", "MKL_NUM_THREADS"):
+        if os.environ.get(kk, "").isdigit():
+            return int(os.environ[kk])
+    return len(os.sched_getaffinity(0))
+
+
+def reference_arm(args):
+    """--impl reference: the oracle on this machine's host cores, same metric and workload."""
+    from exact_tiled_attention_44_b200.inputs import WORKLOADS
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from exact_tiled_attention_44_b200.inputs import make_inputs
+    w = WORKLOADS[args.workload]
+    q, k, v = make_inputs(w)
+    heads = {}
+
+    def head(b, h):
+        if (b, h) not in heads:
+            heads[(b, h)] = _head_arrays(w, q, k, v, b, h)
+        return heads[(b, h)]
+
+    # bounded sample per step: whole query rows of one head, sized so the run ends in minutes
+    t_cal = _oracle_rows_task(head(0, 0) + (w.scale, w.causal, w.window, w.n_sink, w.N - 64, w.N))
+    per_row = max(t_cal / 64, 1e-5)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(w.N, budget / per_row)))
+    step_rows = []
+    for s_ in range(args.warmup + args.steps):
+        b, h = divmod(s_ % (w.B * w.H), w.H)
+        r0 = (s_ * rows) % max(1, w.N - rows + 1)
+        step_rows.append((b, h, r0, r0 + rows))
+    for b, h, r0, r1 in step_rows[:args.warmup]:
+        _oracle_rows_task(head(b, h) + (w.scale, w.causal, w.window, w.n_sink, r0, r1))
+    t0 = time.perf_counter()
+    for b, h, r0, r1 in step_rows[args.warmup:]:
+        _oracle_rows_task(head(b, h) + (w.scale, w.causal, w.window, w.n_sink, r0, r1))
+    wall = time.perf_counter() - t0
+    flops = sum(4.0 * w.d * _pairs_rows(w, r0, r1) for _, _, r0, r1 in step_rows[args.warmup:])
+    value = flops / wall / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} H={w.H} H_kv={w.H_kv} N={w.N} d={w.d} "
+                                   f"{w.dtype} causal={int(w.causal)} window={w.window} "
+                                   f"n_sink={w.n_sink}",
+                       "step": f"{rows} complete query rows of one head per step (bounded sample)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": f"{rows} query rows per step, one head per step, "
+                                       f"float64 numpy, one process"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="c3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import exact_tiled_attention_44_b200 as A
+    from exact_tiled_attention_44_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    w = WORKLOADS[args.workload]
+    q, k, v = make_inputs(w)           # identical seeded inputs on every rank (replicas)
+    sets = []
+    per_set_bytes = 0
+    n_sets = 2
+    for i in range(n_sets):
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        od = torch.empty_like(qd)
+        ld = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        sets.append((qd, kd, vd, od, ld))
+        per_set_bytes = sum(t.numel() * t.element_size() for t in (qd, kd, vd, od, ld))
+    pairs = A.unmasked_pairs(w.N, w.causal, w.window, w.n_sink)
+    flops = 4.0 * w.B * w.H * w.d * pairs
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        qd, kd, vd, od, ld = sets[i % n_sets]
+        A.attention(qd, kd, vd, causal=w.causal, window=w.window, n_sink=w.n_sink, scale=w.scale,
+                    out=od, lse=ld)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0,
+                           os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
+                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    sampler.start()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    n_launch0 = A.launch_count()
+    sampler.mark_begin()
+    t_all0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t_all1.record(stream)
+    barrier()
+    sampler.mark_end()
+    launches = A.launch_count() - n_launch0
+    clocks = sampler.stop()
+    total_ms = t_all0.elapsed_time(t_all1)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * flops * K / (total_ms / 1e3) / 1e12
+    avg_kernel_ms = statistics.mean(kern_ms)
+    achieved = flops / (avg_kernel_ms / 1e3) / 1e12
+
+    # ---- end to end through the public host-buffer entry point
+    e2e_steps = args.e2e_steps or max(3, min(K, 30))
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lh = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+    staging = {"q": sets[0][0], "k": sets[0][1], "v": sets[0][2], "o": sets[0][3], "lse": sets[0][4]}
+    for _ in range(2):
+        A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
+                              window=w.window, n_sink=w.n_sink, scale=w.scale)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
+                              window=w.window, n_sink=w.n_sink, scale=w.scale)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    status = A.get_status()
+
+    if rank == 0:
+        peaks = load_peaks()
+        traffic = load_traffic(w.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} H={w.H} H_kv={w.H_kv} N={w.N} d={w.d} "
+                                   f"{w.dtype} causal={int(w.causal)} window={w.window} "
+                                   f"n_sink={w.n_sink}",
+                       "global_batch": w.B * world, "seq_len": w.N,
+                       "parallelism": f"replicas x{world} (independent problems, no collective)",
+                       "l2": f"inputs larger than L2: {n_sets} rotating device input sets of "
+                             f"{per_set_bytes / 2**20:.0f} MiB (L2 126 MiB)",
+                       "flops_per_step": flops, "kept_pairs_per_head": pairs},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": traffic,
+                         "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"
+                         if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
+                         "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
+                         "kernel_ms": avg_kernel_ms},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "path": "attn_fwd_host: pinned host q,k,v -> device, forward, o and lse -> host"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_throughput(w.name, q, k, v)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,205 @@
+"""Exact tiled attention forward for B200 (sm_100a): Python binding of libattn.so.
+
+Argument marshalling only.  Every arithmetic step of the forward runs in the
+CUDA kernel behind the C ABI declared in ``include/attn.h``; PyTorch supplies
+device memory and streams.  There is no CPU fallback: if the library is not
+built, or the device is not an sm_100 GPU, the calls raise.
+
+    from exact_tiled_attention_44_b200 import attention
+    o, lse = attention(q, k, v, causal=True)          # q,k,v: CUDA bf16/fp16 [B,H,N,d]
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "unmasked_pairs",
+    "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "error_string",
+    "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
+    "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
+    "ATTN_BF16", "ATTN_FP16", "ATTN_OUT_F32",
+]
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_MISALIGNED = -3
+ATTN_ERR_CUDA = -4
+ATTN_ERR_DEVICE_TIMEOUT = -5
+ATTN_BF16 = 0
+ATTN_FP16 = 1
+ATTN_OUT_F32 = 0x10
+
+EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_error_string", "attn_unmasked_pairs",
+                    "attn_visited_blocks", "attn_get_status", "attn_set_watchdog_ns",
+                    "attn_launch_count")
+
+_LIB = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str = "attn_fwd"):
+        self.status = status
+        super().__init__(f"{what} failed: {error_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+
+
+def load_library():
+    """Loads libattn.so (built in-tree); raises if it is missing."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built: run `python -m exact_tiled_attention_44_b200._build`")
+    lib = ctypes.CDLL(path)
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+    lib.attn_fwd.restype = ci
+    lib.attn_fwd_host.argtypes = [vp] * 10 + [ci] * 8 + [cf, ci, vp]
+    lib.attn_fwd_host.restype = ci
+    lib.attn_error_string.argtypes = [ci]
+    lib.attn_error_string.restype = ctypes.c_char_p
+    lib.attn_unmasked_pairs.argtypes = [ci, ci, ci, ci]
+    lib.attn_unmasked_pairs.restype = ctypes.c_longlong
+    lib.attn_visited_blocks.argtypes = [ci, ci, ci, ci]
+    lib.attn_visited_blocks.restype = ctypes.c_longlong
+    lib.attn_get_status.argtypes = []
+    lib.attn_get_status.restype = ci
+    lib.attn_set_watchdog_ns.argtypes = [ctypes.c_ulonglong]
+    lib.attn_set_watchdog_ns.restype = ctypes.c_ulonglong
+    lib.attn_launch_count.argtypes = []
+    lib.attn_launch_count.restype = ctypes.c_ulonglong
+    _LIB = lib
+    return lib
+
+
+def error_string(status: int) -> str:
+    return load_library().attn_error_string(int(status)).decode()
+
+
+def unmasked_pairs(N: int, causal: bool, window: int = 0, n_sink: int = 0) -> int:
+    """Kept (query, key) pairs of one head (host-only helper of the library)."""
+    return int(load_library().attn_unmasked_pairs(N, int(causal), window, n_sink))
+
+
+def visited_blocks(N: int, causal: bool, window: int = 0, n_sink: int = 0) -> int:
+    """128x128 block pairs the kernel's schedule computes for one head."""
+    return int(load_library().attn_visited_blocks(N, int(causal), window, n_sink))
+
+
+def get_status() -> int:
+    """Reads and clears the device watchdog status (synchronises the device)."""
+    return int(load_library().attn_get_status())
+
+
+def set_watchdog_ns(ns: int) -> int:
+    return int(load_library().attn_set_watchdog_ns(int(ns)))
+
+
+def launch_count() -> int:
+    return int(load_library().attn_launch_count())
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) rounded once to float32 (the "HEAD_DIM ** -0.5" of the Hands-On guide)."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float16:
+        return ATTN_FP16
+    raise TypeError(f"q/k/v must be bfloat16 or float16, got {t.dtype}")
+
+
+def attn_fwd_raw(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                 stream) -> int:
+    """Direct C-ABI call with integer pointers; returns the status code."""
+    return int(load_library().attn_fwd(q, k, v, o, lse, B, H, H_kv, N, d, int(causal), window,
+                                       n_sink, ctypes.c_float(scale), dtype, stream))
+
+
+def _check(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, N, d] / [B, H_kv, N, d]")
+    if k.shape != v.shape or q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]:
+        raise ValueError(f"shape mismatch q={tuple(q.shape)} k={tuple(k.shape)} v={tuple(v.shape)}")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    _dtype_code(q)
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
+              window: int = 0, n_sink: int = 0, scale: float | None = None,
+              out_f32: bool = False, out: torch.Tensor | None = None,
+              lse: torch.Tensor | None = None, return_lse: bool = True):
+    """O = softmax(scale * q k^T + mask) v and the per-row natural-log LSE.
+
+    q: [B, H, N, d] CUDA bf16/fp16; k, v: [B, H_kv, N, d] (H % H_kv == 0).
+    Returns (o, lse) with o [B, H, N, d] (float32 when ``out_f32``) and lse
+    [B, H, N] float32 (None when ``return_lse`` is False).
+    """
+    _check(q, k, v)
+    if not q.is_cuda:
+        raise ValueError("attention() takes CUDA tensors; use attention_from_host() for host tensors")
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if scale is None:
+        scale = default_scale(d)
+    code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, B, H, H_kv, N, d, causal,
+                          window, n_sink, scale, code, stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc)
+    return out, lse
+
+
+def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, staging: dict,
+                        out: torch.Tensor, lse: torch.Tensor | None = None, causal: bool = False,
+                        window: int = 0, n_sink: int = 0, scale: float | None = None,
+                        out_f32: bool = False, stream: torch.cuda.Stream | None = None):
+    """Host-resident forward through ``attn_fwd_host``: copies in, computes, copies out.
+
+    q, k, v, out, lse are CPU tensors (page-locked for asynchronous copies);
+    ``staging`` holds device tensors "q", "k", "v", "o" and optionally "lse"
+    of the matching shapes.  Enqueues on ``stream`` (default: current) and
+    returns without synchronising.
+    """
+    _check(q, k, v)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    if scale is None:
+        scale = default_scale(d)
+    code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
+    dev = staging["q"].device
+    s = (stream or torch.cuda.current_stream(dev)).cuda_stream
+    dl = staging.get("lse")
+    with torch.cuda.device(dev):
+        rc = int(load_library().attn_fwd_host(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+            lse.data_ptr() if lse is not None else None,
+            staging["q"].data_ptr(), staging["k"].data_ptr(), staging["v"].data_ptr(),
+            staging["o"].data_ptr(), dl.data_ptr() if dl is not None else None,
+            B, H, H_kv, N, d, int(causal), window, n_sink, ctypes.c_float(scale), code, s))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_host")
+    return out, lse

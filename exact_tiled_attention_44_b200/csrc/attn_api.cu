@@ -1,0 +1,342 @@
+// attn_api.cu -- host side of libattn.so: argument checks, TMA descriptors,
+// persistent-grid launch, and the small host-only helpers of include/attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_kernel.cuh"
+
+namespace {
+
+// Device status word: written by a CTA whose wait timed out, read and cleared
+// by attn_get_status().
+__device__ int g_device_status = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  int* status = nullptr;           // device address of g_device_status
+  uint32_t attr_set = 0;           // one bit per kernel instantiation
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+std::atomic<unsigned long long> g_watchdog_ns{2000000000ull};
+std::atomic<unsigned long long> g_launches{0};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Sizes {
+  size_t q_bytes, kv_bytes, o_bytes, lse_bytes;
+  int elem, d;
+};
+
+// Pure argument validation: touches no CUDA API, so it can be tested on a
+// machine without a GPU.  Returns ATTN_OK and fills `sz` when the call is
+// well formed; `*empty` is set when there is nothing to compute.
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
+             float scale, int dtype, Sizes* sz, bool* empty) {
+  *empty = false;
+  if ((dtype & ~(ATTN_OUT_F32 | 0xF)) != 0) return ATTN_ERR_INVALID_ARG;
+  const int base = dtype & 0xF;
+  if (base != ATTN_BF16 && base != ATTN_FP16) return ATTN_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || N < 0 || H_kv < 1 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (window < 0 || n_sink < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return ATTN_OK;
+  }
+  if (H % H_kv != 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
+  // index ranges: B*H (TMA z extent, unit count) and per-head element counts
+  const long long bh = static_cast<long long>(B) * H;
+  const long long n_pairs = (static_cast<long long>(N) + 2 * attn::BM - 1) / (2 * attn::BM);
+  if (bh > INT32_MAX || bh * n_pairs > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  const int elem = 2;
+  const size_t rows_q = static_cast<size_t>(B) * H * N;
+  const size_t rows_kv = static_cast<size_t>(B) * H_kv * N;
+  sz->elem = elem;
+  sz->d = d;
+  sz->q_bytes = rows_q * d * elem;
+  sz->kv_bytes = rows_kv * d * elem;
+  sz->o_bytes = rows_q * d * ((dtype & ATTN_OUT_F32) ? 4 : elem);
+  sz->lse_bytes = rows_q * sizeof(float);
+  if (overlaps(o, sz->o_bytes, q, sz->q_bytes) || overlaps(o, sz->o_bytes, k, sz->kv_bytes) ||
+      overlaps(o, sz->o_bytes, v, sz->kv_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse != nullptr &&
+      (overlaps(lse, sz->lse_bytes, q, sz->q_bytes) || overlaps(lse, sz->lse_bytes, k, sz->kv_bytes) ||
+       overlaps(lse, sz->lse_bytes, v, sz->kv_bytes) || overlaps(lse, sz->lse_bytes, o, sz->o_bytes)))
+    return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&st.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&st.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (st.cc_major != 10 || st.cc_minor != 0) return ATTN_ERR_UNSUPPORTED;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return ATTN_ERR_CUDA;
+    st.status = static_cast<int*>(addr);
+    if (g_encode == nullptr) {
+      cudaDriverEntryPointQueryResult qres;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) !=
+              cudaSuccess ||
+          qres != cudaDriverEntryPointSuccess || fn == nullptr)
+        return ATTN_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    st.ready = true;
+  }
+  *out = &st;
+  return ATTN_OK;
+}
+
+// 3-D view [z][rows][d] of a contiguous [.., N, d] tensor; box = (cw, 128, 1)
+// with the swizzle span equal to the box's row bytes.
+int encode_map(CUtensorMap* map, const void* base, bool bf16, int d, int n, int z) {
+  const int cw = d < 64 ? d : 64;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                              static_cast<cuuint64_t>(z)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(n) * d * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(cw), 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = cw * 2 == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : cw * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                              3, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool BF16, bool F32>
+int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
+               const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
+  auto kern = attn::attn_fwd_kernel<D, BF16, F32>;
+  const int smem = attn::Geo<D>::SMEM_BYTES + 1024;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!(st->attr_set & (1u << bit))) {
+      // The kernel re-splits its registers between warpgroups after launch;
+      // that only works when every thread starts with LAUNCH_REGS registers.
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (fa.numRegs < attn::LAUNCH_REGS) return ATTN_ERR_UNSUPPORTED;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      st->attr_set |= 1u << bit;
+    }
+  }
+  const int grid = kp.num_units < st->sm_count ? kp.num_units : st->sm_count;
+  kern<<<grid, attn::NUM_THREADS, smem, stream>>>(mq, mk, mv, kp);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+int launch_d(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
+             const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
+  const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
+  const int bit = dbit * 4 + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
+  if (bf16)
+    return f32 ? launch_one<D, true, true>(st, bit, mq, mk, mv, kp, stream)
+               : launch_one<D, true, false>(st, bit, mq, mk, mv, kp, stream);
+  return f32 ? launch_one<D, false, true>(st, bit, mq, mk, mv, kp, stream)
+             : launch_one<D, false, false>(st, bit, mq, mk, mv, kp, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int H_kv, int N, int d, int causal, int window, int n_sink, float scale, int dtype,
+             void* stream) {
+  Sizes sz;
+  bool empty = false;
+  int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype, &sz,
+                    &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+
+  const bool bf16 = (dtype & 0xF) == ATTN_BF16;
+  const bool f32 = (dtype & ATTN_OUT_F32) != 0;
+  alignas(64) CUtensorMap mq, mk, mv;
+  if (encode_map(&mq, q, bf16, d, N, B * H) != ATTN_OK ||
+      encode_map(&mk, k, bf16, d, N, B * H_kv) != ATTN_OK ||
+      encode_map(&mv, v, bf16, d, N, B * H_kv) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+
+  attn::KernelParams kp;
+  kp.o = o;
+  kp.lse = lse;
+  kp.status = st->status;
+  kp.watchdog_ns = g_watchdog_ns.load(std::memory_order_relaxed);
+  kp.B = B;
+  kp.H = H;
+  kp.H_kv = H_kv;
+  kp.N = N;
+  kp.causal = causal;
+  // A window at least as long as the sequence keeps every causal key.
+  kp.window = (window >= N) ? 0 : window;
+  kp.n_sink = kp.window > 0 ? (n_sink < N ? n_sink : N) : 0;
+  kp.scale_log2 = scale * 1.4426950408889634f;
+  kp.n_qpairs = (N + 2 * attn::BM - 1) / (2 * attn::BM);
+  kp.n_kblocks = (N + attn::BN - 1) / attn::BN;
+  kp.num_units = B * H * kp.n_qpairs;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 16: return launch_d<16>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 32: return launch_d<32>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 64: return launch_d<64>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 128: return launch_d<128>(st, bf16, f32, mq, mk, mv, kp, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, void* dq,
+                  void* dk, void* dv, void* dout, float* dlse, int B, int H, int H_kv, int N,
+                  int d, int causal, int window, int n_sink, float scale, int dtype,
+                  void* stream) {
+  Sizes sz;
+  bool empty = false;
+  int rc = validate(dq, dk, dv, dout, dlse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                    &sz, &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q, sz.q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, sz.kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, sz.kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  rc = attn_fwd(dq, dk, dv, dout, dlse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                stream);
+  if (rc != ATTN_OK) return rc;
+  if (cudaMemcpyAsync(o, dout, sz.o_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (lse != nullptr && dlse != nullptr &&
+      cudaMemcpyAsync(lse, dlse, sz.lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+const char* attn_error_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case ATTN_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "kernel wait exceeded the watchdog limit";
+    default: return "unknown status";
+  }
+}
+
+long long attn_unmasked_pairs(int N, int causal, int window, int n_sink) {
+  if (N < 0 || window < 0 || n_sink < 0 || (causal != 0 && causal != 1)) return -1;
+  if (window > 0 && !causal) return -1;
+  const long long n = N;
+  if (!causal) return n * n;
+  if (window == 0 || window >= N) return n * (n + 1) / 2;
+  // Row i keeps min(i+1, W) window keys plus the sinks left of its window:
+  // max(0, min(S, i - W + 1)).
+  const long long W = window, S = n_sink;
+  long long total = 0;
+  // window part: rows 0..W-1 keep i+1, rows W..N-1 keep W
+  total += W * (W + 1) / 2 + (n - W) * W;
+  // sink part: rows i >= W contribute min(S, i - W + 1)
+  const long long rows = n - W;                   // i - W + 1 runs over 1..rows
+  const long long full = rows > S ? rows - S : 0; // rows where the count is S
+  const long long ramp = rows - full;             // counts 1..ramp
+  total += ramp * (ramp + 1) / 2 + full * S;
+  return total;
+}
+
+long long attn_visited_blocks(int N, int causal, int window, int n_sink) {
+  if (N < 0 || window < 0 || n_sink < 0 || (causal != 0 && causal != 1)) return -1;
+  if (window > 0 && !causal) return -1;
+  if (N == 0) return 0;
+  const int W = (window >= N) ? 0 : window;
+  const int S = W > 0 ? (n_sink < N ? n_sink : N) : 0;
+  const int nkb = (N + attn::BN - 1) / attn::BN;
+  const int sink_blocks = W > 0 ? (S + attn::BN - 1) / attn::BN : 0;
+  long long total = 0;
+  for (int r0 = 0; r0 < N; r0 += attn::BM) {
+    const int r_last = (r0 + attn::BM - 1 < N - 1) ? r0 + attn::BM - 1 : N - 1;
+    int lo = 0, hi = nkb;
+    if (causal) hi = (r_last / attn::BN + 1 < nkb) ? r_last / attn::BN + 1 : nkb;
+    if (W > 0) {
+      const int k_min = r0 - W + 1;
+      lo = k_min > 0 ? k_min / attn::BN : 0;
+    }
+    const int tsb = sink_blocks < hi ? sink_blocks : hi;
+    const int win_start = lo > tsb ? lo : tsb;
+    total += tsb + (hi > win_start ? hi - win_start : 0);
+  }
+  return total;
+}
+
+int attn_get_status(void) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  int value = 0;
+  const int zero = 0;
+  if (cudaMemcpy(&value, st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return value;
+}
+
+unsigned long long attn_set_watchdog_ns(unsigned long long ns) {
+  if (ns < 1000000ull) ns = 1000000ull;
+  if (ns > 60000000000ull) ns = 60000000000ull;
+  return g_watchdog_ns.exchange(ns);
+}
+
+unsigned long long attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,717 @@
+// attn_kernel.cuh -- exact tiled attention forward for sm_100a.
+//
+// What it computes (per batch b, query head h, kv head g = h / (H / H_kv)):
+//   O = softmax(scale * Q K^T + mask) V  and  LSE = ln sum_kept exp(scale q.k),
+// tile by tile with the online softmax of "Tiled attention with online
+// softmax" (Lab 3) and "USAAIO Lesson 91" slide 11: per query row a running
+// max m, a running denominator l and an output accumulator rescaled by
+// exp(m_old - m_new) when the max grows; O is divided by l and written to HBM
+// once at the end ("Flash Attention", dileepadev: "Write output once").  The
+// N x N score matrix never leaves the chip: each 128 x 128 score tile lives in
+// tensor memory (TMEM) only.
+//
+// Layout of one CTA (persistent; one CTA per SM, 384 threads):
+//   warps 0-3  softmax warpgroup for Q tile 0 (TMEM lanes 0-127 = its rows)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp 8     MMA issue (one thread) + TMEM allocation
+//   warp 9     TMA producer (one thread)
+//   warps 10-11 idle (they hand their registers to the softmax warpgroups)
+// A work unit is (b, h, a pair of adjacent 128-row Q tiles).  Both Q tiles
+// consume the same K/V block stream, so every K/V block loaded from HBM feeds
+// two 128 x 128 x d MMAs per GEMM.
+//
+// Per K/V block j and Q tile t:
+//   MMA warp   S_t = Q_t K_j^T         (tcgen05.mma, A and B from smem, fp32 in TMEM)
+//   softmax t  reads S_t row-per-thread (tcgen05.ld 32x32b), masks boundary
+//              blocks, updates m and l, writes P_t = exp2(s*scale*log2e - m)
+//              as 16-bit over the first half of S_t's columns, and rescales
+//              O_t in TMEM when the max grew by more than 2^8 (lazy rescale:
+//              otherwise the stale max is kept; exact, because O and l share it)
+//   MMA warp   O_t += P_t V_j          (tcgen05.mma, A from TMEM, B from smem)
+// The MMA warp interleaves the two Q tiles so that one tile's softmax overlaps
+// the other tile's MMAs.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace attn {
+
+constexpr int BM = 128;           // query rows per Q tile
+constexpr int BN = 128;           // keys per K/V block
+constexpr int NUM_STAGES = 2;     // K ring depth (and V ring depth)
+constexpr int NUM_THREADS = 384;           // three warpgroups
+constexpr int MMA_WARP = 8;
+constexpr int TMA_WARP = 9;
+// Register split after launch: the two softmax warpgroups grow to 208 per
+// thread, the MMA/TMA warpgroup shrinks to 88.  The launch must give every
+// thread at least LAUNCH_REGS so that 256 * 208 + 128 * 88 fits the block's
+// allocation (384 * 168 = 64512); the host checks this before launching.
+constexpr uint32_t SOFTMAX_REGS = 208;
+constexpr uint32_t CONTROL_REGS = 88;
+constexpr int LAUNCH_REGS = 168;
+static_assert(256 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split exceeds the launch allocation");
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale when the max grows by > 256x
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int STATUS_TIMEOUT = -5;         // matches ATTN_ERR_DEVICE_TIMEOUT
+
+struct KernelParams {
+  void* o;
+  float* lse;
+  int* status;
+  unsigned long long watchdog_ns;
+  int B, H, H_kv, N;
+  int causal, window, n_sink;
+  float scale_log2;   // scale * log2(e)
+  int n_qpairs;       // ceil(N / 256)
+  int n_kblocks;      // ceil(N / 128)
+  int num_units;      // B * H * n_qpairs
+};
+
+// Shared-memory geometry for head dimension D (16-bit elements).  A 128 x D
+// tile is stored as D / CW column chunks of 128 rows x CB bytes, each chunk in
+// the TMA / tcgen05 swizzle of span CB (32, 64 or 128 bytes).
+template <int D>
+struct Geo {
+  static constexpr int CW = D < 64 ? D : 64;
+  static constexpr int CB = CW * 2;
+  static constexpr int NCH = D / CW;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int CHUNK_BYTES = 128 * CB;
+  // descriptor layout field: 6 = 32B swizzle, 4 = 64B, 2 = 128B
+  static constexpr uint32_t LAYOUT = CB == 128 ? 2u : (CB == 64 ? 4u : 6u);
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + NUM_STAGES * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + NUM_STAGES * TILE_BYTES;
+  static constexpr int SMEM_BYTES = BAR_OFF + 256;
+  static constexpr uint32_t S_COL0 = 0;      // S_t at column 128 t
+  static constexpr uint32_t O_COL0 = 256;    // O_t at column 256 + D t
+  static_assert(D % 16 == 0 && D <= 128, "unsupported head dim");
+  static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
+};
+
+// Barrier slots (8 bytes each) after the tiles.
+enum BarSlot : int {
+  B_Q_FULL = 0, B_Q_EMPTY = 1,
+  B_K_FULL = 2, B_K_EMPTY = B_K_FULL + NUM_STAGES,
+  B_V_FULL = B_K_EMPTY + NUM_STAGES, B_V_EMPTY = B_V_FULL + NUM_STAGES,
+  B_S_FULL = B_V_EMPTY + NUM_STAGES,   // [2]
+  B_P_FULL = B_S_FULL + 2,             // [2]
+  B_O_FULL = B_P_FULL + 2,             // [2]
+  B_DRAIN = B_O_FULL + 2,
+  B_COUNT = B_DRAIN + 1
+};
+constexpr int TMEM_SLOT_OFF = 8 * B_COUNT;
+constexpr int ABORT_FLAG_OFF = TMEM_SLOT_OFF + 4;
+
+// ------------------------------------------------------------ descriptors
+
+// tcgen05 shared-memory matrix descriptor: start address, leading and stride
+// byte offsets (16-byte units), fixed version bits 46-47 = 1, swizzle mode in
+// bits 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator (bits 4-5 = 1), A and B
+// format (bits 7-9, 10-12: 0 = f16, 1 = bf16), B major-ness (bit 16: 1 = MN
+// major), N / 8 (bits 17-22), M / 16 (bits 24-28).
+__host__ __device__ constexpr uint32_t instr_desc(bool bf16, int m, int n, bool b_mn_major) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------ schedule
+
+// One work unit: query rows [q0, q0 + 256) of head (b, h).  Key blocks are
+// iterated as a sink prefix [0, sb) followed by [wlo, hi_max); Q tile t uses
+// block j iff j < sb_t or lo_t <= j < hi_t.  Blocks holding no kept
+// pair for a tile are skipped ("Tiled attention with online softmax": only key
+// blocks at or before the query block; exercise 4: sinks and a window).
+struct Unit {
+  int bh, b, h, g, q0;
+  int n_active;
+  int sb, wlo, n_iter;
+  int sb0, lo0, hi0, sb1, lo1, hi1;   // per Q tile: sink prefix, window range
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
+  Unit U;
+  const int BH = p.B * p.H;
+  // Longest-processing-time first: causal cost grows with the pair index, so
+  // units are handed out from the last pair of every head down to the first.
+  const int pair = p.n_qpairs - 1 - u / BH;
+  U.bh = u % BH;
+  U.b = U.bh / p.H;
+  U.h = U.bh % p.H;
+  U.g = U.h / (p.H / p.H_kv);
+  U.q0 = pair * 2 * BM;
+  U.n_active = (U.q0 + BM < p.N) ? 2 : 1;
+  const int sink_blocks = (p.window > 0) ? (p.n_sink + BN - 1) / BN : 0;
+  int sb = 0, lo_min = 1 << 30, hi_max = 0;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = U.q0 + t * BM;
+    const int r_last = min(r0 + BM - 1, p.N - 1);
+    int lo = 0, hi = p.n_kblocks;
+    if (p.causal) hi = min(p.n_kblocks, r_last / BN + 1);
+    if (p.window > 0) {
+      const int k_min = r0 - p.window + 1;
+      lo = k_min > 0 ? k_min / BN : 0;
+    }
+    const int tsb = min(sink_blocks, hi);
+    if (t == 0) {
+      U.sb0 = tsb; U.lo0 = lo; U.hi0 = hi;
+    } else {
+      U.sb1 = tsb; U.lo1 = lo; U.hi1 = hi;
+    }
+    if (t < U.n_active) {
+      sb = max(sb, tsb);
+      lo_min = min(lo_min, lo);
+      hi_max = max(hi_max, hi);
+    }
+  }
+  U.sb = sb;
+  U.wlo = max(lo_min, sb);
+  U.n_iter = sb + max(0, hi_max - U.wlo);
+  return U;
+}
+
+__device__ __forceinline__ int block_at(const Unit& U, int idx) {
+  return idx < U.sb ? idx : U.wlo + (idx - U.sb);
+}
+
+__device__ __forceinline__ bool tile_uses(const Unit& U, int t, int j) {
+  const int sb = t == 0 ? U.sb0 : U.sb1;
+  const int lo = t == 0 ? U.lo0 : U.lo1;
+  const int hi = t == 0 ? U.hi0 : U.hi1;
+  return t < U.n_active && (j < sb || (j >= lo && j < hi));
+}
+
+__device__ __forceinline__ int tile_last_block(const Unit& U, int t) {
+  return (t == 0 ? U.hi0 : U.hi1) - 1;
+}
+
+// True when some (row, key) of Q tile rows [r0, r0+128) x keys [c0, c0+128)
+// is masked, so the element mask must be applied.
+__device__ __forceinline__ bool block_needs_mask(const KernelParams& p, int r0, int c0) {
+  if (c0 + BN > p.N) return true;
+  if (p.causal && c0 + BN - 1 > r0) return true;
+  if (p.window > 0 && !(r0 + BM - 1 - c0 < p.window) && !(c0 + BN <= p.n_sink)) return true;
+  return false;
+}
+
+__device__ __forceinline__ bool kept(const KernelParams& p, int i, int j) {
+  if (j >= p.N) return false;
+  if (p.causal && j > i) return false;
+  if (p.window > 0 && !(i - j < p.window || j < p.n_sink)) return false;
+  return true;
+}
+
+// ------------------------------------------------------------ watchdog wait
+
+// Waits for `parity` on `bar`.  Gives up when another role has aborted or when
+// the wait exceeds the watchdog limit; the first to time out records the
+// status and raises the CTA's abort flag.  Returns false on give-up.
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* status, unsigned long long limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicExch(status, STATUS_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, const KernelParams& p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag, p.status, p.watchdog_ns);
+}
+
+// Bounded wait used while draining after an abort (no status update).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
+                                           unsigned long long limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return;
+  }
+}
+
+// Two floats -> one 32-bit word of two 16-bit values (round to nearest
+// even), the first in the low half.
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h2);
+  } else {
+    __half2 h2 = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h2);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float unpack_lo(uint32_t w) {
+  if constexpr (BF16) return __uint_as_float(w << 16);
+  else return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+}
+
+template <bool BF16>
+__device__ __forceinline__ float unpack_hi(uint32_t w) {
+  if constexpr (BF16) return __uint_as_float(w & 0xFFFF0000u);
+  else return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+template <int W>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[W]) {
+  if constexpr (W == 32) tmem_ld_32x32b_x32(taddr, r);
+  else tmem_ld_32x32b_x16(taddr, r);
+}
+
+template <int W>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[W]) {
+  if constexpr (W == 32) tmem_st_32x32b_x32(taddr, r);
+  else tmem_st_32x32b_x16(taddr, r);
+  tmem_wait_st();
+}
+
+// ------------------------------------------------------------ roles
+
+template <int D>
+__device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                         const CUtensorMap* tmV, uint32_t sbase, uint32_t bars,
+                         volatile int* abort_flag) {
+  using G = Geo<D>;
+  uint32_t q_it = 0, kv_it = 0;
+  // parity of the last load issued into each barrier, for the drain
+  int q_last = -1, k_last[NUM_STAGES], v_last[NUM_STAGES];
+  for (int s = 0; s < NUM_STAGES; ++s) k_last[s] = v_last[s] = -1;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    const Unit U = decode_unit(u, p);
+    ok = wait_or_abort(bars + 8 * B_Q_EMPTY, (q_it & 1u) ^ 1u, abort_flag, p);
+    if (!ok) break;
+    mbar_arrive_expect_tx(bars + 8 * B_Q_FULL, U.n_active * G::TILE_BYTES);
+    for (int t = 0; t < U.n_active; ++t)
+      for (int c = 0; c < G::NCH; ++c)
+        tma_load_3d(sbase + G::Q_OFF + t * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
+                    bars + 8 * B_Q_FULL, c * G::CW, U.q0 + t * BM, U.bh);
+    q_last = q_it & 1;
+    ++q_it;
+    const int kvz = U.b * p.H_kv + U.g;
+    for (int idx = 0; idx < U.n_iter; ++idx, ++kv_it) {
+      const int j = block_at(U, idx);
+      const int s = kv_it % NUM_STAGES;
+      const uint32_t ph = (kv_it / NUM_STAGES) & 1u;
+      ok = wait_or_abort(bars + 8 * (B_K_EMPTY + s), ph ^ 1u, abort_flag, p);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * (B_K_FULL + s), G::TILE_BYTES);
+      for (int c = 0; c < G::NCH; ++c)
+        tma_load_3d(sbase + G::K_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmK,
+                    bars + 8 * (B_K_FULL + s), c * G::CW, j * BN, kvz);
+      k_last[s] = ph;
+      ok = wait_or_abort(bars + 8 * (B_V_EMPTY + s), ph ^ 1u, abort_flag, p);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * (B_V_FULL + s), G::TILE_BYTES);
+      for (int c = 0; c < G::NCH; ++c)
+        tma_load_3d(sbase + G::V_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmV,
+                    bars + 8 * (B_V_FULL + s), c * G::CW, j * BN, kvz);
+      v_last[s] = ph;
+    }
+  }
+  if (!ok) {
+    // Let every copy this thread started land before the CTA can exit.
+    const unsigned long long lim = p.watchdog_ns;
+    if (q_last >= 0) drain_wait(bars + 8 * B_Q_FULL, q_last, lim);
+    for (int s = 0; s < NUM_STAGES; ++s) {
+      if (k_last[s] >= 0) drain_wait(bars + 8 * (B_K_FULL + s), k_last[s], lim);
+      if (v_last[s] >= 0) drain_wait(bars + 8 * (B_V_FULL + s), v_last[s], lim);
+    }
+  }
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int t, int stage) {
+  using G = Geo<D>;
+  constexpr uint32_t idesc = instr_desc(BF16, BM, BN, false);
+  const uint32_t qa = sbase + G::Q_OFF + t * G::TILE_BYTES;
+  const uint32_t ka = sbase + G::K_OFF + stage * G::TILE_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    // K-major operands: 16 elements (32 bytes) per step inside a swizzle row;
+    // the next chunk starts CHUNK_BYTES later.  Stride between 8-row groups is
+    // 8 * CB; the leading offset is unused for swizzled K-major layouts.
+    const uint32_t off = (kk * 16 / G::CW) * G::CHUNK_BYTES + ((kk * 16) % G::CW) * 2;
+    const uint64_t da = smem_desc(qa + off, 16, 8 * G::CB, G::LAYOUT);
+    const uint64_t db = smem_desc(ka + off, 16, 8 * G::CB, G::LAYOUT);
+    mma_ss(tmem + Geo<D>::S_COL0 + t * BN, da, db, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int t, int stage,
+                                         bool accumulate) {
+  using G = Geo<D>;
+  constexpr uint32_t idesc = instr_desc(BF16, BM, D, true);
+  const uint32_t va = sbase + G::V_OFF + stage * G::TILE_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    // A = P: 16 keys per step = 8 packed 32-bit TMEM columns.
+    // B = V, MN-major: 16 key rows per step (16 * CB bytes); 8-row groups are
+    // 8 * CB apart (stride offset); column chunks are CHUNK_BYTES apart
+    // (leading offset).
+    const uint64_t db = smem_desc(va + kk * 16 * G::CB, G::CHUNK_BYTES, 8 * G::CB, G::LAYOUT);
+    mma_ts(tmem + G::O_COL0 + t * D, tmem + G::S_COL0 + t * BN + kk * 8, db, idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool BF16>
+__device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, uint32_t bars,
+                         volatile int* abort_flag) {
+  uint32_t q_ph = 0, kv_it = 0, p_ph[2] = {0, 0};
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    const Unit U = decode_unit(u, p);
+    ok = wait_or_abort(bars + 8 * B_Q_FULL, q_ph, abort_flag, p);
+    if (!ok) break;
+    q_ph ^= 1u;
+    tc_fence_after_sync();
+    // prologue: S_t for the first block
+    {
+      const int j0 = block_at(U, 0);
+      const int s = kv_it % NUM_STAGES;
+      ok = wait_or_abort(bars + 8 * (B_K_FULL + s), (kv_it / NUM_STAGES) & 1u, abort_flag, p);
+      if (!ok) break;
+      tc_fence_after_sync();
+      for (int t = 0; t < 2; ++t)
+        if (tile_uses(U, t, j0)) {
+          issue_qk<D, BF16>(tmem, sbase, t, s);
+          mma_commit(bars + 8 * (B_S_FULL + t));
+        }
+      mma_commit(bars + 8 * (B_K_EMPTY + s));
+      if (U.n_iter == 1) mma_commit(bars + 8 * B_Q_EMPTY);
+    }
+    int pv_done[2] = {0, 0};
+    for (int idx = 0; idx < U.n_iter && ok; ++idx) {
+      const int j = block_at(U, idx);
+      const uint32_t it = kv_it + idx;
+      const int s = it % NUM_STAGES;
+      ok = wait_or_abort(bars + 8 * (B_V_FULL + s), (it / NUM_STAGES) & 1u, abort_flag, p);
+      if (!ok) break;
+      const bool has_next = idx + 1 < U.n_iter;
+      const int jn = has_next ? block_at(U, idx + 1) : 0;
+      const uint32_t itn = it + 1;
+      const int sn = itn % NUM_STAGES;
+      // Q tile 0: P0 V_j, then S0 for the next block
+      if (tile_uses(U, 0, j)) {
+        ok = wait_or_abort(bars + 8 * (B_P_FULL + 0), p_ph[0], abort_flag, p);
+        if (!ok) break;
+        p_ph[0] ^= 1u;
+        tc_fence_after_sync();
+        issue_pv<D, BF16>(tmem, sbase, 0, s, pv_done[0] > 0);
+        ++pv_done[0];
+        if (j == tile_last_block(U, 0)) mma_commit(bars + 8 * (B_O_FULL + 0));
+      }
+      if (has_next) {
+        ok = wait_or_abort(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (tile_uses(U, 0, jn)) {
+          issue_qk<D, BF16>(tmem, sbase, 0, sn);
+          mma_commit(bars + 8 * (B_S_FULL + 0));
+        }
+      }
+      // Q tile 1: P1 V_j, then S1 for the next block
+      if (tile_uses(U, 1, j)) {
+        ok = wait_or_abort(bars + 8 * (B_P_FULL + 1), p_ph[1], abort_flag, p);
+        if (!ok) break;
+        p_ph[1] ^= 1u;
+        tc_fence_after_sync();
+        issue_pv<D, BF16>(tmem, sbase, 1, s, pv_done[1] > 0);
+        ++pv_done[1];
+        if (j == tile_last_block(U, 1)) mma_commit(bars + 8 * (B_O_FULL + 1));
+      }
+      mma_commit(bars + 8 * (B_V_EMPTY + s));
+      if (has_next) {
+        if (tile_uses(U, 1, jn)) {
+          issue_qk<D, BF16>(tmem, sbase, 1, sn);
+          mma_commit(bars + 8 * (B_S_FULL + 1));
+        }
+        mma_commit(bars + 8 * (B_K_EMPTY + sn));
+        if (idx + 2 == U.n_iter) mma_commit(bars + 8 * B_Q_EMPTY);
+      }
+    }
+    kv_it += U.n_iter;
+  }
+  // Every MMA this thread issued has completed once the drain barrier flips.
+  mma_commit(bars + 8 * B_DRAIN);
+  drain_wait(bars + 8 * B_DRAIN, 0, p.watchdog_ns);
+}
+
+template <int D, bool BF16, bool OUT_F32>
+__device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars, int t,
+                             int warp_in_wg, int lane, volatile int* abort_flag) {
+  using G = Geo<D>;
+  constexpr int OC = D >= 32 ? 32 : 16;   // TMEM columns per O load/store
+  const int row_in_tile = warp_in_wg * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(warp_in_wg * 32) << 16;
+  const uint32_t s_tmem = tmem + lane_base + G::S_COL0 + t * BN;
+  const uint32_t o_tmem = tmem + lane_base + G::O_COL0 + t * D;
+  const float c = p.scale_log2;
+  uint32_t s_ph = 0, o_ph = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    const Unit U = decode_unit(u, p);
+    if (t >= U.n_active) continue;
+    const int r0 = U.q0 + t * BM;
+    const int row = r0 + row_in_tile;
+    float m_run = -INFINITY, l_exact = 0.f, l_round = 0.f;
+    bool first = true;
+    for (int idx = 0; idx < U.n_iter; ++idx) {
+      const int j = block_at(U, idx);
+      if (!tile_uses(U, t, j)) continue;
+      ok = wait_or_abort(bars + 8 * (B_S_FULL + t), s_ph, abort_flag, p);
+      if (!ok) break;
+      s_ph ^= 1u;
+      tc_fence_after_sync();
+      uint32_t sr[128];
+      tmem_ld_32x32b_x128(s_tmem, sr);
+      const int c0 = j * BN;
+      const bool masked = block_needs_mask(p, r0, c0);
+      float m_blk;
+      if (masked) {
+        // Scale first, then drop masked keys with -inf (any sign of scale).
+        // Kept keys of this row, in block-local columns e = j - c0:
+        //   e <= hi (causal limit and key padding) and (e >= lo (window) or e < sk (sinks))
+        const int hi = (p.causal ? min(row, p.N - 1) : p.N - 1) - c0;
+        const int lo = p.window > 0 ? row - p.window + 1 - c0 : -(1 << 30);
+        const int sk = p.window > 0 ? p.n_sink - c0 : -(1 << 30);
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const float x = __uint_as_float(sr[e]) * c;
+          const bool keep = (e <= hi) && (e >= lo || e < sk);
+          sr[e] = __float_as_uint(keep ? x : -INFINITY);
+        }
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 128; e += 4) {
+          m0 = max3(m0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+          m1 = max3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+        }
+        m_blk = fmaxf(m0, m1);
+      } else {
+        // raw-score extreme, then one multiply: max of s*c is c*max(s) for c >= 0
+        // and c*min(s) for c < 0
+        float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
+        if (c >= 0.f) {
+#pragma unroll
+          for (int e = 2; e < 126; e += 4) {
+            m0 = max3(m0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            m1 = max3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+          }
+          m0 = max3(m0, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+          m_blk = fmaxf(m0, m1) * c;
+        } else {
+#pragma unroll
+          for (int e = 2; e < 126; e += 4) {
+            m0 = min3(m0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            m1 = min3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+          }
+          m0 = min3(m0, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+          m_blk = fminf(m0, m1) * c;
+        }
+      }
+      // online softmax update (log2 units); lazy rescale
+      const float m_new = fmaxf(m_run, m_blk);
+      float alpha = 1.f;
+      const bool rescale = m_new > m_run + RESCALE_THRESHOLD;
+      if (rescale) {
+        alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+      const float2 cc2 = masked ? make_float2(1.f, 1.f) : make_float2(c, c);
+      const float2 nm2 = make_float2(-mref, -mref);
+      // Two denominators: le sums the fp32 weights (for the LSE), lr sums the
+      // same 16-bit-rounded weights the P V MMA consumes (for O, so that every
+      // output row is a convex combination of V rows under those weights).
+      float2 le = make_float2(0.f, 0.f), lr = make_float2(0.f, 0.f);
+      // P in four 32-key chunks: 16 packed words each, stored as soon as they
+      // are ready so that the score registers are released chunk by chunk.
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+        float2 le_q = make_float2(0.f, 0.f), lr_q = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 x = make_float2(__uint_as_float(sr[32 * q4 + 2 * e]),
+                                       __uint_as_float(sr[32 * q4 + 2 * e + 1]));
+          const float2 a = fma2(x, cc2, nm2);
+          const float2 pe = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+          pk[e] = pack2<BF16>(pe.x, pe.y);
+          le_q = add2(le_q, pe);
+          lr_q = add2(lr_q, make_float2(unpack_lo<BF16>(pk[e]), unpack_hi<BF16>(pk[e])));
+        }
+        tmem_st_32x32b_x16(s_tmem + 16 * q4, pk);
+        le = add2(le, le_q);
+        lr = add2(lr, lr_q);
+      }
+      l_exact = l_exact * alpha + (le.x + le.y);
+      l_round = l_round * alpha + (lr.x + lr.y);
+      // O_t holds the previous blocks' sum (the MMA that produced S_t for this
+      // block was issued after the previous P_t V, so that PV has completed).
+      if (!first && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int cc = 0; cc < D / OC; ++cc) {
+          uint32_t orr[OC];
+          tmem_ld_cols<OC>(o_tmem + cc * OC, orr);
+#pragma unroll
+          for (int e = 0; e < OC; e += 2) {
+            const float2 r2 = mul2(make_float2(__uint_as_float(orr[e]), __uint_as_float(orr[e + 1])),
+                                   make_float2(alpha, alpha));
+            orr[e] = __float_as_uint(r2.x);
+            orr[e + 1] = __float_as_uint(r2.y);
+          }
+          tmem_st_cols<OC>(o_tmem + cc * OC, orr);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (B_P_FULL + t));
+      first = false;
+    }
+    if (!ok) break;
+    // epilogue: O = O_acc / l, written once; LSE = (m + log2 l) ln 2
+    ok = wait_or_abort(bars + 8 * (B_O_FULL + t), o_ph, abort_flag, p);
+    if (!ok) break;
+    o_ph ^= 1u;
+    tc_fence_after_sync();
+    const float inv_l = 1.f / l_round;
+    const bool valid = row < p.N;
+    const size_t row_off = (static_cast<size_t>(U.bh) * p.N + row) * D;
+#pragma unroll
+    for (int cc = 0; cc < D / OC; ++cc) {
+      uint32_t orr[OC];
+      tmem_ld_cols<OC>(o_tmem + cc * OC, orr);
+      if (valid) {
+        if constexpr (OUT_F32) {
+          float* dst = reinterpret_cast<float*>(p.o) + row_off + cc * OC;
+#pragma unroll
+          for (int e = 0; e < OC; e += 4) {
+            const float4 v4 = make_float4(
+                __uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l,
+                __uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
+            *reinterpret_cast<float4*>(dst + e) = v4;
+          }
+        } else {
+          uint32_t packed[OC / 2];
+#pragma unroll
+          for (int e = 0; e < OC / 2; ++e)
+            packed[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
+                                    __uint_as_float(orr[2 * e + 1]) * inv_l);
+          uint16_t* dst = reinterpret_cast<uint16_t*>(p.o) + row_off + cc * OC;
+#pragma unroll
+          for (int e = 0; e < OC / 2; e += 4)
+            *reinterpret_cast<uint4*>(dst + 2 * e) =
+                make_uint4(packed[e], packed[e + 1], packed[e + 2], packed[e + 3]);
+        }
+      }
+    }
+    if (valid && p.lse != nullptr)
+      p.lse[static_cast<size_t>(U.bh) * p.N + row] = (m_run + __log2f(l_exact)) * 0.69314718055994531f;
+  }
+}
+
+template <int D, bool BF16, bool OUT_F32>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const KernelParams p) {
+  using G = Geo<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment keeps every tile on a swizzle-pattern boundary.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bars = sbase + G::BAR_OFF;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + G::BAR_OFF + ABORT_FLAG_OFF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::BAR_OFF + TMEM_SLOT_OFF);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars + 8 * B_Q_FULL, 1);
+    mbar_init(bars + 8 * B_Q_EMPTY, 1);
+    for (int s = 0; s < NUM_STAGES; ++s) {
+      mbar_init(bars + 8 * (B_K_FULL + s), 1);
+      mbar_init(bars + 8 * (B_K_EMPTY + s), 1);
+      mbar_init(bars + 8 * (B_V_FULL + s), 1);
+      mbar_init(bars + 8 * (B_V_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bars + 8 * (B_S_FULL + t), 1);
+      mbar_init(bars + 8 * (B_P_FULL + t), 4);   // one arrival per softmax warp
+      mbar_init(bars + 8 * (B_O_FULL + t), 1);
+    }
+    mbar_init(bars + 8 * B_DRAIN, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == TMA_WARP && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  // Each branch ends on its own copy of the final barrier: code shared by
+  // warps running under different register budgets would have to fit the
+  // smaller one.
+  if (warp < 8) {
+    regs_increase<SOFTMAX_REGS>();
+    softmax_role<D, BF16, OUT_F32>(p, tmem, bars, warp / 4, warp % 4, lane, abort_flag);
+    tc_fence_before_sync();
+    __syncthreads();
+  } else {
+    regs_decrease<CONTROL_REGS>();
+    if (warp == MMA_WARP) {
+      if (lane == 0) mma_role<D, BF16>(p, tmem, sbase, bars, abort_flag);
+    } else if (warp == TMA_WARP) {
+      if (lane == 0) tma_role<D>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, TMEM_COLS);
+    }
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,152 @@
+/*
+ * attn.h -- C ABI of the exact tiled attention forward library (libattn.so).
+ *
+ * The library computes, for every batch b and query head h,
+ *
+ *     O[b,h]   = softmax(scale * Q[b,h] K[b,g]^T + mask) V[b,g]
+ *     LSE[b,h] = log-sum-exp (natural log) of the same masked, scaled logits
+ *
+ * with g = h / (H / H_kv), tile by tile with the online softmax (a running row
+ * max m, a running denominator l and a rescaled output accumulator), never
+ * materialising the N x N score matrix.  Sources of the definition:
+ *   - "Flash Attention" (dileepadev learn-ai), "The Problem with Standard
+ *     Attention" (the formula) and "Mathematical Equivalence" (the tiled form
+ *     gives the same result, it is not an approximation); "Write output once".
+ *   - "Tiled attention with online softmax" (Lab 3): the causal tiled loop
+ *     with running max, running denominator and running numerator, key blocks
+ *     after the query block skipped; exercise 4 (sinks + sliding window).
+ *   - "USAAIO Lesson 91", slide 11 (the tiled update equations) and slide 32
+ *     (MQA / GQA: query heads share K/V heads).
+ *   - "Hands-On Build Guide: Flash Attention ... in NumPy", Step 2 (causal
+ *     mask: key j is kept for query i iff j <= i) and Step 5 (a log-sum-exp
+ *     carried across tiles).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are contiguous, row-major.  q and o are [B, H, N, d];
+ *     k and v are [B, H_kv, N, d]; lse is [B, H, N] float32.
+ *   - The mask keeps key j for query i iff
+ *       (!causal || j <= i) && (window == 0 || i - j < window || j < n_sink).
+ *     window counts the query itself (window = 1 keeps only the diagonal);
+ *     sink keys are positions 0 .. n_sink-1 and stay subject to causality.
+ *   - LSE_i = ln( sum over kept j of exp(scale * q_i . k_j) ).
+ *   - The library never allocates device or host memory in these calls; the
+ *     caller owns every buffer.
+ *   - Every call returns an attn_status_t.  Argument errors are detected
+ *     before anything is enqueued.  Calls are asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream);
+ *     faults inside the kernel surface at the caller's next synchronisation,
+ *     and watchdog expiries are reported by attn_get_status().
+ *   - Results are deterministic: equal inputs give bitwise-equal outputs.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,     /* a size, pointer or flag is out of range   */
+  ATTN_ERR_UNSUPPORTED = -2,     /* valid request this build does not handle  */
+  ATTN_ERR_MISALIGNED = -3,      /* a tensor pointer is not 16-byte aligned    */
+  ATTN_ERR_CUDA = -4,            /* a CUDA runtime/driver call failed          */
+  ATTN_ERR_DEVICE_TIMEOUT = -5   /* a kernel wait exceeded its time limit      */
+} attn_status_t;
+
+/* dtype argument: element type of q, k, v (and o), optionally OR-ed with
+ * ATTN_OUT_F32 to make o float32 (the fp32 accumulator divided by l, before
+ * any 16-bit rounding). */
+enum {
+  ATTN_BF16 = 0,
+  ATTN_FP16 = 1,
+  ATTN_OUT_F32 = 0x10
+};
+
+/*
+ * attn_fwd -- exact masked attention forward on device buffers.
+ *
+ *   q      device, [B, H, N, d] bf16/fp16 (dtype), 16-byte aligned, read only
+ *   k, v   device, [B, H_kv, N, d], same element type, 16-byte aligned
+ *   o      device, [B, H, N, d]: same element type, or float32 when
+ *          dtype & ATTN_OUT_F32; 16-byte aligned; must not overlap q, k or v
+ *   lse    device, [B, H, N] float32, or NULL to skip writing it
+ *   B, H, H_kv, N   sizes; B, H, N >= 0 (any zero: nothing to do, ATTN_OK,
+ *          pointers may then be NULL); H_kv >= 1 and H % H_kv == 0
+ *   d      head dimension: 16, 32, 64 or 128 (else ATTN_ERR_UNSUPPORTED)
+ *   causal 0 or 1
+ *   window 0 (none) or >= 1 keys including the query itself; needs causal
+ *          (window > 0 with causal == 0 is ATTN_ERR_UNSUPPORTED)
+ *   n_sink >= 0 always-kept leading keys; only meaningful with window > 0
+ *   scale  finite float multiplying q.k before masking (0 is allowed)
+ *   dtype  ATTN_BF16 or ATTN_FP16, optionally | ATTN_OUT_F32
+ *   stream cudaStream_t as void*
+ *
+ * Needs an sm_100 device (B200); other devices give ATTN_ERR_UNSUPPORTED.
+ * Returns after the kernel is enqueued.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
+             float scale, int dtype, void* stream);
+
+/*
+ * attn_fwd_host -- the same forward for HOST-resident inputs and outputs.
+ *
+ * Enqueues on `stream`: host->device copies of q, k, v into the caller's
+ * device staging buffers dq, dk, dv; attn_fwd(dq, dk, dv, dout, dlse, ...);
+ * device->host copies of dout into o and (when both are non-NULL) dlse into
+ * lse.  Host buffers should be page-locked for the copies to be
+ * asynchronous.  The caller synchronises `stream` before reading o / lse.
+ * Sizes, flags and errors are those of attn_fwd; every pointer must be
+ * 16-byte aligned.
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                  void* dq, void* dk, void* dv, void* dout, float* dlse,
+                  int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
+                  float scale, int dtype, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* attn_error_string(int status);
+
+/*
+ * attn_unmasked_pairs -- host only: the number of kept (query, key) pairs of
+ * one head under the mask rule above (N*N non-causal, N(N+1)/2 causal).  This
+ * is the work the FLOP count 4*d*pairs credits ("Tiled attention with online
+ * softmax", exercise 3 compares visited work with the full n^2).  Returns -1
+ * for invalid arguments.
+ */
+long long attn_unmasked_pairs(int N, int causal, int window, int n_sink);
+
+/*
+ * attn_visited_blocks -- host only: the number of (128-query-row block,
+ * 128-key block) pairs the kernel's schedule computes for one head.  A block
+ * pair is visited iff it holds at least one kept pair (causal, window and sink
+ * skipping as in Lab 3's "only key blocks at or before this query block").
+ * Returns -1 for invalid arguments.
+ */
+long long attn_visited_blocks(int N, int causal, int window, int n_sink);
+
+/*
+ * attn_get_status -- reads and clears the device status word of the current
+ * device.  Every wait inside the kernel is bounded (about attn_watchdog_ns
+ * nanoseconds); a CTA whose wait expires drains its own in-flight copies and
+ * tensor-core work, releases its tensor memory, records
+ * ATTN_ERR_DEVICE_TIMEOUT here and returns.  Synchronises the device.
+ */
+int attn_get_status(void);
+
+/* Sets the watchdog limit in nanoseconds for later launches on every device
+ * (default 2e9, clamped to [1e6, 6e10]).  Returns the previous value. */
+unsigned long long attn_set_watchdog_ns(unsigned long long ns);
+
+/* Number of kernel launches enqueued by this process so far (all entry
+ * points).  Lets a caller count the GPU launches of a region. */
+unsigned long long attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,133 @@
+"""C-ABI boundary on the CPU: the library loads, exports what include/attn.h
+declares, rejects malformed calls before touching CUDA, and its host-only
+schedule helpers agree with the oracle's mask."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import exact_tiled_attention_44_b200 as A
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+# Fake, 16-byte aligned, never dereferenced addresses (validation runs first).
+P_Q, P_K, P_V, P_O, P_L = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = A.load_library()
+    decl = declared_functions()
+    assert decl == sorted(A.EXPORTED_SYMBOLS)
+    for name in decl:
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_error_strings():
+    for code in (A.ATTN_OK, A.ATTN_ERR_INVALID_ARG, A.ATTN_ERR_UNSUPPORTED, A.ATTN_ERR_MISALIGNED,
+                 A.ATTN_ERR_CUDA, A.ATTN_ERR_DEVICE_TIMEOUT, 12345):
+        assert isinstance(A.error_string(code), str) and A.error_string(code)
+
+
+def call(q=P_Q, k=P_K, v=P_V, o=P_O, lse=P_L, B=1, H=2, H_kv=2, N=100, d=64, causal=1, window=0,
+         n_sink=0, scale=0.125, dtype=A.ATTN_BF16):
+    return A.attn_fwd_raw(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                          None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=-1), A.ATTN_ERR_INVALID_ARG),
+    (dict(N=-5), A.ATTN_ERR_INVALID_ARG),
+    (dict(H_kv=0), A.ATTN_ERR_INVALID_ARG),
+    (dict(H=6, H_kv=4), A.ATTN_ERR_INVALID_ARG),
+    (dict(d=0), A.ATTN_ERR_INVALID_ARG),
+    (dict(d=48), A.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), A.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=2), A.ATTN_ERR_INVALID_ARG),
+    (dict(window=-1), A.ATTN_ERR_INVALID_ARG),
+    (dict(n_sink=-1), A.ATTN_ERR_INVALID_ARG),
+    (dict(causal=0, window=8), A.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), A.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), A.ATTN_ERR_INVALID_ARG),
+    (dict(dtype=2), A.ATTN_ERR_INVALID_ARG),
+    (dict(dtype=0x20), A.ATTN_ERR_INVALID_ARG),
+    (dict(q=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(o=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(q=P_Q + 8), A.ATTN_ERR_MISALIGNED),
+    (dict(v=P_V + 2), A.ATTN_ERR_MISALIGNED),
+    (dict(lse=P_L + 4), A.ATTN_ERR_MISALIGNED),
+    (dict(o=P_Q + 64), A.ATTN_ERR_INVALID_ARG),          # o overlaps q
+    (dict(o=P_K), A.ATTN_ERR_INVALID_ARG),               # o aliases k
+    (dict(lse=P_O + 16), A.ATTN_ERR_INVALID_ARG),        # lse overlaps o
+])
+def test_invalid_calls_are_rejected_before_launch(kw, expect):
+    assert call(**kw) == expect
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(N=0),
+                                dict(B=0, q=None, k=None, v=None, o=None, lse=None)])
+def test_empty_problem_is_a_no_op(kw):
+    assert call(**kw) == A.ATTN_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 1, 8, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        A.attention(q, q, q)
+    with pytest.raises(TypeError):
+        A.attention(q.float(), q.float(), q.float())
+
+
+@pytest.mark.parametrize("N,causal,window,n_sink", [
+    (1, 1, 0, 0), (1, 0, 0, 0), (7, 0, 0, 0), (64, 1, 0, 0), (1000, 1, 0, 0),
+    (300, 1, 1, 0), (300, 1, 17, 5), (777, 1, 128, 64), (777, 1, 300, 200), (257, 1, 256, 0),
+    (200, 1, 500, 10), (1024, 1, 1024, 64), (1500, 1, 129, 130)])
+def test_unmasked_pairs_matches_oracle_enumeration(N, causal, window, n_sink):
+    assert A.unmasked_pairs(N, causal, window, n_sink) == oracle.kept_pairs(N, bool(causal), window, n_sink)
+
+
+def test_unmasked_pairs_workloads():
+    assert A.unmasked_pairs(4096, 1) == 4096 * 4097 // 2
+    assert A.unmasked_pairs(1024, 0) == 1024 * 1024
+    assert A.unmasked_pairs(8192, 1, 1024, 64) == 8321568
+    assert A.unmasked_pairs(10, 0, 3, 0) == -1
+    assert A.unmasked_pairs(-1, 1) == -1
+
+
+def _visited_by_mask(N, causal, window, n_sink, blk=128):
+    keep = oracle.keep_mask(N, N, bool(causal), window, n_sink)
+    nb = (N + blk - 1) // blk
+    count = 0
+    for qb in range(nb):
+        for kb in range(nb):
+            if keep[qb * blk:(qb + 1) * blk, kb * blk:(kb + 1) * blk].any():
+                count += 1
+    return count
+
+
+@pytest.mark.parametrize("N,causal,window,n_sink", [
+    (1, 1, 0, 0), (64, 1, 0, 0), (64, 0, 0, 0), (200, 1, 0, 0), (1000, 0, 0, 0),
+    (1000, 1, 0, 0), (1000, 1, 1, 0), (1000, 1, 100, 0), (1000, 1, 300, 64),
+    (1300, 1, 129, 200), (1300, 1, 257, 1), (900, 1, 2000, 5)])
+def test_visited_blocks_is_exactly_the_blocks_with_kept_pairs(N, causal, window, n_sink):
+    """Lab 3, exercise 3: count visited block pairs; none is skipped that holds work."""
+    assert A.visited_blocks(N, causal, window, n_sink) == _visited_by_mask(N, causal, window, n_sink)
+
+
+def test_visited_blocks_workloads():
+    assert A.visited_blocks(4096, 1) == 528           # 32 * 33 / 2
+    assert A.visited_blocks(1024, 0) == 64
+    assert A.visited_blocks(1024, 1) == 36
+    assert A.visited_blocks(16384, 1) == 128 * 129 // 2
+    assert A.visited_blocks(64, 1) == 1

@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded, 16-bit-rounded inputs, plus oracle-free invariants."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_tiled_attention_44_b200 as A
+from exact_tiled_attention_44_b200.inputs import WORKLOADS, make_inputs, random_qkv, to_f64
+from parity_utils import (assert_parity, errors, oracle_full, oracle_rows, round_floor, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+BF, FP = torch.bfloat16, torch.float16
+
+# (B, H, H_kv, N, d, dtype, causal, window, n_sink)
+SWEEP = [
+    (1, 1, 1, 1, 64, BF, 1, 0, 0),
+    (1, 1, 1, 1, 128, FP, 0, 0, 0),
+    (1, 1, 1, 7, 16, BF, 1, 0, 0),
+    (1, 2, 1, 63, 128, BF, 1, 0, 0),
+    (1, 1, 1, 64, 16, BF, 0, 0, 0),
+    (2, 2, 2, 65, 64, FP, 1, 0, 0),
+    (1, 3, 1, 127, 32, BF, 0, 0, 0),
+    (1, 1, 1, 128, 128, BF, 1, 0, 0),
+    (1, 2, 2, 129, 128, FP, 0, 0, 0),
+    (1, 2, 2, 200, 64, FP, 1, 0, 0),
+    (2, 4, 2, 255, 128, BF, 1, 0, 0),
+    (1, 2, 1, 256, 32, FP, 1, 0, 0),
+    (1, 2, 2, 257, 16, BF, 0, 0, 0),
+    (1, 2, 2, 384, 128, BF, 0, 0, 0),
+    (1, 4, 4, 500, 64, BF, 1, 0, 0),
+    (1, 2, 1, 640, 128, FP, 1, 0, 0),
+    (1, 1, 1, 1100, 128, BF, 1, 0, 0),
+    (1, 2, 2, 500, 128, BF, 1, 1, 0),
+    (1, 2, 2, 500, 64, BF, 1, 100, 0),
+    (1, 2, 1, 700, 128, BF, 1, 130, 3),
+    (1, 2, 2, 900, 128, FP, 1, 128, 64),
+    (1, 1, 1, 900, 32, BF, 1, 300, 200),
+    (1, 2, 2, 300, 128, BF, 1, 1000, 5),
+    (1, 2, 1, 1000, 16, BF, 1, 257, 129),
+    (2, 8, 1, 600, 128, BF, 1, 256, 64),
+]
+
+
+def _id(c):
+    B, H, Hk, N, d, dt, ca, w, s = c
+    return f"B{B}H{H}k{Hk}N{N}d{d}{'bf' if dt == BF else 'fp'}{'c' if ca else 'n'}w{w}s{s}"
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=[_id(c) for c in SWEEP])
+def test_sweep_full_parity(case):
+    B, H, Hk, N, d, dt, causal, window, n_sink = case
+    q, k, v = random_qkv(B, H, Hk, N, d, dt, seed=N * 131 + d)
+    scale = A.default_scale(d)
+    Or, Lr = oracle_full(q, k, v, bool(causal), window, n_sink, scale)
+    o32, l32 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=True)
+    assert_parity(errors(o32, l32, Or, Lr), what="fp32 out")
+    o16, l16 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=False)
+    assert o16.dtype == dt
+    assert_parity(errors(o16, l16, Or, Lr), round_floor(Or, dt), what="16-bit out")
+    # the 16-bit output is the fp32 output rounded once
+    assert torch.equal(o16, o32.to(dt))
+    assert torch.equal(l16, l32)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.2, 0.9, 3.0])
+def test_scale_values(scale):
+    q, k, v = random_qkv(1, 2, 2, 300, 64, BF, seed=7)
+    for causal in (True, False):
+        Or, Lr = oracle_full(q, k, v, causal, 0, 0, scale)
+        o, l = run_gpu(q, k, v, causal, 0, 0, scale, out_f32=True)
+        assert_parity(errors(o, l, Or, Lr), what=f"scale={scale} causal={causal}")
+
+
+def test_large_logits_rescale():
+    """Logit ranges far beyond the lazy-rescale threshold (std 4 inputs, scale 1)."""
+    q, k, v = random_qkv(1, 2, 2, 777, 128, BF, seed=11, std=2.0)
+    Or, Lr = oracle_full(q, k, v, True, 0, 0, 0.5)
+    o, l = run_gpu(q, k, v, True, 0, 0, 0.5, out_f32=True)
+    assert_parity(errors(o, l, Or, Lr), what="large logits")
+
+
+# --------------------------------------------------------------- workloads
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c2c"])
+def test_small_workloads_full(name):
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    Or, Lr = oracle_full(q, k, v, w.causal, w.window, w.n_sink, w.scale)
+    o32, l32 = run_gpu(q, k, v, w.causal, w.window, w.n_sink, w.scale, out_f32=True)
+    assert_parity(errors(o32, l32, Or, Lr), what=name)
+    o16, l16 = run_gpu(q, k, v, w.causal, w.window, w.n_sink, w.scale, out_f32=False)
+    assert_parity(errors(o16, l16, Or, Lr), round_floor(Or, w.torch_dtype), what=name + " 16-bit")
+
+
+def _sample_rows(N, rng, extra=24):
+    base = [0, 1, 2, 63, 64, 127, 128, 129, 255, 256, 257, 1023, 1024, 1025, N // 2,
+            N - 257, N - 256, N - 129, N - 128, N - 2, N - 1]
+    rows = sorted(set([r for r in base if 0 <= r < N] + list(rng.integers(0, N, extra))))
+    return np.array(rows)
+
+
+@pytest.mark.parametrize("name", ["c3", "c4", "c5"])
+def test_full_size_workloads_sampled(name):
+    """Full-size launch (as bench.py times it); oracle on sampled rows of several heads."""
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o32, l32 = A.attention(qd, kd, vd, causal=w.causal, window=w.window, n_sink=w.n_sink,
+                           scale=w.scale, out_f32=True)
+    o16, l16 = A.attention(qd, kd, vd, causal=w.causal, window=w.window, n_sink=w.n_sink,
+                           scale=w.scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o32).all() and torch.isfinite(l32).all()
+    assert torch.equal(o16, o32.to(w.torch_dtype))
+    rng = np.random.default_rng(0)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 3)]
+    for b, h in heads:
+        rows = _sample_rows(w.N, rng)
+        Or, Lr = oracle_rows(q, k, v, b, h, rows, w.causal, w.window, w.n_sink, w.scale)
+        idx = torch.from_numpy(rows).cuda()
+        err = errors(o32[b, h, idx], l32[b, h, idx], Or, Lr)
+        assert_parity(err, what=f"{name} head ({b},{h})")
+        err16 = errors(o16[b, h, idx], None, Or, Lr)
+        assert_parity(err16, round_floor(Or, w.torch_dtype), what=f"{name} 16-bit ({b},{h})")
+
+
+# --------------------------------------------------------- oracle-free checks
+
+def test_causal_row0_is_v0_exactly():
+    q, k, v = random_qkv(2, 3, 3, 300, 128, BF, seed=3)
+    o, l = run_gpu(q, k, v, True, 0, 0, 0.3, out_f32=True)
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0].float())
+    expect = 0.3 * (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1)
+    assert (l[:, :, 0].double().cpu() - expect).abs().max() < 1e-3
+
+
+@pytest.mark.parametrize("causal,window,n_sink", [(True, 0, 0), (False, 0, 0), (True, 200, 70)])
+def test_identical_keys_give_mean_of_kept_values(causal, window, n_sink):
+    B, H, N, d = 1, 2, 700, 64
+    q, _, v = random_qkv(B, H, H, N, d, BF, seed=5)
+    k = torch.randn(d, generator=torch.Generator().manual_seed(9)).to(BF).expand(B, H, N, d).contiguous()
+    o, l = run_gpu(q, k, v, causal, window, n_sink, 0.125, out_f32=True)
+    import oracle as orc
+    keep = orc.keep_mask(N, N, causal, window, n_sink)
+    V = to_f64(v)
+    ref = np.einsum("ij,bhjd->bhid", keep / keep.sum(1, keepdims=True), V)
+    assert np.abs(o.double().cpu().numpy() - ref).max() < 1e-2
+    s = 0.125 * (to_f64(q) @ to_f64(k)[0, 0, 0])
+    assert np.abs(l.double().cpu().numpy() - (s + np.log(keep.sum(1)))).max() < 1e-3
+
+
+def test_mqa_equals_repeated_mha_bitwise():
+    B, H, Hk, N, d = 2, 8, 2, 520, 128
+    q, k, v = random_qkv(B, H, Hk, N, d, BF, seed=13)
+    o1, l1 = run_gpu(q, k, v, True, 0, 0, 0.088, out_f32=True)
+    kr, vr = k.repeat_interleave(H // Hk, 1).contiguous(), v.repeat_interleave(H // Hk, 1).contiguous()
+    o2, l2 = run_gpu(q, kr, vr, True, 0, 0, 0.088, out_f32=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_deterministic_bitwise():
+    w = WORKLOADS["c2c"]
+    q, k, v = make_inputs(w)
+    a = run_gpu(q, k, v, True, 0, 0, w.scale, out_f32=False)
+    b = run_gpu(q, k, v, True, 0, 0, w.scale, out_f32=False)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_noncausal_key_permutation():
+    q, k, v = random_qkv(1, 2, 2, 400, 64, FP, seed=17)
+    perm = torch.randperm(400, generator=torch.Generator().manual_seed(1))
+    o1, l1 = run_gpu(q, k, v, False, 0, 0, 0.125, out_f32=True)
+    o2, l2 = run_gpu(q, k[:, :, perm].contiguous(), v[:, :, perm].contiguous(), False, 0, 0, 0.125,
+                     out_f32=True)
+    assert (o1 - o2).abs().max() < 1e-2 and (l1 - l2).abs().max() < 1e-3
+
+
+def test_no_quadratic_workspace():
+    """The library allocates nothing: memory around a long-sequence call is the outputs only."""
+    q, k, v = (t.cuda() for t in random_qkv(1, 4, 4, 8192, 128, BF, seed=1))
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 4, 8192, device="cuda")
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    before = torch.cuda.memory_allocated()
+    A.attention(q, k, v, causal=True, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == before
+
+
+def test_host_entry_point_matches_device():
+    w = WORKLOADS["c2c"]
+    q, k, v = make_inputs(w)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lh = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+    staging = {"q": torch.empty_like(q, device="cuda"), "k": torch.empty_like(k, device="cuda"),
+               "v": torch.empty_like(v, device="cuda"), "o": torch.empty_like(q, device="cuda"),
+               "lse": torch.empty(q.shape[:3], device="cuda")}
+    A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    o, l = run_gpu(q, k, v, True, 0, 0, w.scale, out_f32=False)
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, l.cpu())
+
+
+def test_side_stream_and_launch_count():
+    q, k, v = (t.cuda() for t in random_qkv(1, 2, 2, 333, 64, BF, seed=2))
+    ref, lref = A.attention(q, k, v, causal=True)
+    s = torch.cuda.Stream()
+    n0 = A.launch_count()
+    with torch.cuda.stream(s):
+        o, l = A.attention(q, k, v, causal=True)
+    s.synchronize()
+    assert A.launch_count() == n0 + 1
+    assert torch.equal(o, ref) and torch.equal(l, lref)
+    assert A.get_status() == 0
+
+
+def test_lse_optional():
+    q, k, v = (t.cuda() for t in random_qkv(1, 1, 1, 200, 64, BF, seed=4))
+    o1, _ = A.attention(q, k, v, causal=True, return_lse=False)
+    o2, _ = A.attention(q, k, v, causal=True)
+    assert torch.equal(o1, o2)
