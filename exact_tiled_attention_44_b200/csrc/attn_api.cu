@@ -149,7 +149,10 @@ template <int D, bool BF16, bool F32>
 int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
                const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
   auto kern = attn::attn_fwd_kernel<D, BF16, F32>;
-  const int smem = attn::Geo<D>::SMEM_BYTES + 1024;
+  // At least half of the SM's shared memory, so that two CTAs can never share
+  // an SM (each allocates all 512 TMEM columns).
+  const int smem_need = attn::Geo<D>::SMEM_BYTES + 1024;
+  const int smem = smem_need > 120 * 1024 ? smem_need : 120 * 1024;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!(st->attr_set & (1u << bit))) {

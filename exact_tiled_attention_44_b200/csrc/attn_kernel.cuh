@@ -187,6 +187,20 @@ __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
   return U;
 }
 
+// Work units handed to CTA `cta` of `grid`: round r takes unit r*grid + cta
+// on even rounds and r*grid + (grid - 1 - cta) on odd rounds.  With units in
+// descending cost order this "snake" assignment evens out the per-CTA totals
+// (plain round robin gives the low-numbered CTAs the larger unit of every
+// round).  Returns -1 when the CTA has no unit in round r.
+__device__ __forceinline__ int unit_of_round(int r, int cta, int grid, int num_units) {
+  const int u = r * grid + ((r & 1) ? (grid - 1 - cta) : cta);
+  return u < num_units ? u : -1;
+}
+
+__device__ __forceinline__ int num_rounds(int grid, int num_units) {
+  return (num_units + grid - 1) / grid;
+}
+
 __device__ __forceinline__ int block_at(const Unit& U, int idx) {
   return idx < U.sb ? idx : U.wlo + (idx - U.sb);
 }
@@ -304,7 +318,10 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
   int q_last = -1, k_last[NUM_STAGES], v_last[NUM_STAGES];
   for (int s = 0; s < NUM_STAGES; ++s) k_last[s] = v_last[s] = -1;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  const int rounds = num_rounds(gridDim.x, p.num_units);
+  for (int r = 0; r < rounds && ok; ++r) {
+    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
+    if (u < 0) continue;
     const Unit U = decode_unit(u, p);
     ok = wait_or_abort(bars + 8 * B_Q_EMPTY, (q_it & 1u) ^ 1u, abort_flag, p);
     if (!ok) break;
@@ -388,7 +405,10 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
                          volatile int* abort_flag) {
   uint32_t q_ph = 0, kv_it = 0, p_ph[2] = {0, 0};
   bool ok = true;
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  const int rounds = num_rounds(gridDim.x, p.num_units);
+  for (int r = 0; r < rounds && ok; ++r) {
+    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
+    if (u < 0) continue;
     const Unit U = decode_unit(u, p);
     ok = wait_or_abort(bars + 8 * B_Q_FULL, q_ph, abort_flag, p);
     if (!ok) break;
@@ -478,7 +498,10 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
   const float c = p.scale_log2;
   uint32_t s_ph = 0, o_ph = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  const int rounds = num_rounds(gridDim.x, p.num_units);
+  for (int r = 0; r < rounds && ok; ++r) {
+    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
+    if (u < 0) continue;
     const Unit U = decode_unit(u, p);
     if (t >= U.n_active) continue;
     const int r0 = U.q0 + t * BM;

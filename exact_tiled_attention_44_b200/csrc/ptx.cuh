@@ -72,6 +72,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d) : "memory");
+}
+
+// Orders this thread's earlier shared-memory stores before later reads of
+// that memory by the async proxy (the tensor core).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 // Whole-warp: allocates `ncols` TMEM columns, writes the base address to smem.
@@ -236,6 +248,32 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 va, vb, vd;\n\t"
+      "mov.b64 va, {%2, %3};\n\tmov.b64 vb, {%4, %5};\n\t"
+      "sub.rn.f32x2 vd, va, vb;\n\tmov.b64 {%0, %1}, vd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// acc += lo16(w) + hi16(w), with w holding two bf16 (or f16) values; fp32
+// accumulate, one rounding per add.
+__device__ __forceinline__ float add_bf16x2_to_f32(float acc, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+      : "+f"(acc) : "r"(w));
+  return acc;
+}
+
+__device__ __forceinline__ float add_f16x2_to_f32(float acc, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+      : "+f"(acc) : "r"(w));
+  return acc;
 }
 
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
