@@ -169,8 +169,9 @@ def cpu_oracle_throughput(name: str, q, k, v, budget_s: float = 20.0):
 
     Chunks of complete query rows of distinct heads are spread over all host
     cores (one BLAS thread per worker process, spawn start method; the parent
-    sends each worker only the head it needs).  Returns the cpu_baseline
-    object in TFLOP/s.
+    sends each worker only the head it needs).  New chunks are submitted until
+    ``budget_s`` seconds have passed; the throughput counts the chunks that
+    finished.  Returns the cpu_baseline object in TFLOP/s.
     """
     import concurrent.futures as cf
     import multiprocessing as mp
@@ -178,9 +179,7 @@ def cpu_oracle_throughput(name: str, q, k, v, budget_s: float = 20.0):
     w = WORKLOADS[name]
     cores = len(os.sched_getaffinity(0))
     rows_per_task = 256
-    saved = {kk: os.environ.get(kk) for kk in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
-    for kk in saved:
-        os.environ[kk] = "1"
+    n_chunks = (w.N + rows_per_task - 1) // rows_per_task
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     arrays = {}
 
@@ -188,19 +187,35 @@ def cpu_oracle_throughput(name: str, q, k, v, budget_s: float = 20.0):
         b, h = heads[i % len(heads)]
         if (b, h) not in arrays:
             arrays[(b, h)] = _head_arrays(w, q, k, v, b, h)
-        n_chunks = (w.N + rows_per_task - 1) // rows_per_task
         r0 = ((i // len(heads)) * 7 % n_chunks) * rows_per_task
-        return arrays[(b, h)] + (w.scale, w.causal, w.window, w.n_sink, r0, min(w.N, r0 + rows_per_task))
+        return arrays[(b, h)] + (w.scale, w.causal, w.window, w.n_sink, r0,
+                                 min(w.N, r0 + rows_per_task))
 
+    saved = {kk: os.environ.get(kk) for kk in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for kk in saved:
+        os.environ[kk] = "1"
+    done_rows = []
     try:
         ctx = mp.get_context("spawn")
         with cf.ProcessPoolExecutor(max_workers=cores, mp_context=ctx) as ex:
-            cal = [task(i) for i in range(min(cores, 4))]
-            per_task = max(1e-3, statistics.median(ex.map(_oracle_rows_task, cal)))
-            n_tasks = max(cores, int(budget_s * cores / per_task))
-            tasks = [task(i) for i in range(n_tasks)]
+            list(ex.map(_oracle_rows_task, [task(0)] * cores))      # start the workers
             t0 = time.perf_counter()
-            list(ex.map(_oracle_rows_task, tasks, chunksize=max(1, n_tasks // (4 * cores))))
+            nxt = 0
+            pending = {}
+            for _ in range(2 * cores):
+                args = task(nxt)
+                pending[ex.submit(_oracle_rows_task, args)] = args
+                nxt += 1
+            while pending:
+                finished, _ = cf.wait(pending, return_when=cf.FIRST_COMPLETED)
+                for f in finished:
+                    args = pending.pop(f)
+                    f.result()
+                    done_rows.append((args[7], args[8]))
+                    if time.perf_counter() - t0 < budget_s:
+                        a2 = task(nxt)
+                        pending[ex.submit(_oracle_rows_task, a2)] = a2
+                        nxt += 1
             wall = time.perf_counter() - t0
     finally:
         for kk, val in saved.items():
@@ -208,11 +223,11 @@ def cpu_oracle_throughput(name: str, q, k, v, budget_s: float = 20.0):
                 os.environ.pop(kk, None)
             else:
                 os.environ[kk] = val
-    flops = sum(4.0 * w.d * _pairs_rows(w, t[7], t[8]) for t in tasks)
+    flops = sum(4.0 * w.d * _pairs_rows(w, r0, r1) for r0, r1 in done_rows)
     return {"value": flops / wall / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(tasks)} chunks of {rows_per_task} complete query rows from the "
-                      f"{w.B * w.H} heads of {name}; float64 full score rows; {wall:.1f} s wall "
-                      f"on {cores} worker processes"}
+            "sample": f"{len(done_rows)} chunks of {rows_per_task} complete query rows from the "
+                      f"{w.B * w.H} heads of {name} (submitted for {budget_s:.0f} s); float64 full "
+                      f"score rows; {wall:.1f} s wall on {cores} worker processes"}
 
 
 def _blas_threads() -> int:
@@ -274,6 +289,23 @@ def reference_arm(args):
     return 0
 
 
+# ----------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, dist_mod, device) -> float:
+    """Maximum of a per-rank float over all ranks (identity without a process group)."""
+    if dist_mod is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_step: float, steps: int, ms: float) -> float:
+    """Weak scaling: every rank runs the same-size workload; the job rate counts all ranks."""
+    return world * flops_per_step * steps / (ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def main():
@@ -285,6 +317,7 @@ def main():
     ap.add_argument("--workload", default="c3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--clocks-csv", default=None, help="keep the raw nvidia-smi samples here")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -338,8 +371,7 @@ def main():
     barrier()
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0,
-                           os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
-                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+                           f"{args.clocks_csv}.r{rank}" if args.clocks_csv else None)
     sampler.start()
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -359,12 +391,9 @@ def main():
     clocks = sampler.stop()
     total_ms = t_all0.elapsed_time(t_all1)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / K
-    value = world * flops * K / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(world, flops, K, total_ms)
     avg_kernel_ms = statistics.mean(kern_ms)
     achieved = flops / (avg_kernel_ms / 1e3) / 1e12
 
@@ -386,11 +415,8 @@ def main():
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = whole_job_tflops(world, flops, e2e_steps, e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 

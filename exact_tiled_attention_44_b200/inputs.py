@@ -6,7 +6,7 @@ float64 oracle consume exactly the tensors produced here (the oracle takes
 their exact float64 upcast).
 
 Workloads (shapes and mask settings of the pages' examples, scaled to B200
-sizes; the recipe is restated in the design doc):
+sizes):
 
 * ``c1``: one causal head, B=1 H=1 N=64 d=16, scale 1/sqrt(16), bf16.  The draw
   is the one "Tiled attention with online softmax" (Lab 3) makes: one

@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = -1,     /* a size, pointer or flag is out of range   */
-  ATTN_ERR_UNSUPPORTED = -2,     /* valid request this build does not handle  */
+  ATTN_ERR_UNSUPPORTED = -2,     /* valid request this library does not handle */
   ATTN_ERR_MISALIGNED = -3,      /* a tensor pointer is not 16-byte aligned    */
   ATTN_ERR_CUDA = -4,            /* a CUDA runtime/driver call failed          */
   ATTN_ERR_DEVICE_TIMEOUT = -5   /* a kernel wait exceeded its time limit      */

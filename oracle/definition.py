@@ -22,7 +22,7 @@ pages state that the tiled method reaches that definition exactly:
 * "USAAIO Lesson 91", slide 32 (MQA: H query heads share one K/V head; GQA:
   G groups of query heads share one K/V head each).
 
-Readings taken where the pages are open (each is listed in the design doc):
+Readings taken where the pages are open:
 
 * keep(i, j) = (not causal or j <= i) and (window == 0 or i - j < window or
   j < n_sink).  The window counts the query itself; sink keys are the first
