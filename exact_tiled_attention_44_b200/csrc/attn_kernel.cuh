@@ -13,8 +13,8 @@
 // Layout of one CTA (persistent; one CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup for Q tile 0 (TMEM lanes 0-127 = its rows)
 //   warps 4-7  softmax warpgroup for Q tile 1
-//   warp 8     MMA issue (one thread) + TMEM allocation
-//   warp 9     TMA producer (one thread)
+//   warp 8     MMA issue (whole warp, one elected lane issues) + TMEM allocation
+//   warp 9     TMA producer (whole warp, one elected lane issues)
 //   warps 10-11 idle (they hand their registers to the softmax warpgroups)
 // A work unit is (b, h, a pair of adjacent 128-row Q tiles).  Both Q tiles
 // consume the same K/V block stream, so every K/V block loaded from HBM feeds
@@ -259,6 +259,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
   return wait_slow(bar, parity, abort_flag, p.status, p.watchdog_ns);
 }
 
+// wait_or_abort for a whole converged warp; every lane gets the same verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          const KernelParams& p) {
+  const bool ok = wait_or_abort(bar, parity, abort_flag, p);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used while draining after an abort (no status update).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
                                            unsigned long long limit_ns) {
@@ -323,13 +330,16 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     const Unit U = decode_unit(u, p);
-    ok = wait_or_abort(bars + 8 * B_Q_EMPTY, (q_it & 1u) ^ 1u, abort_flag, p);
+    ok = warp_wait(bars + 8 * B_Q_EMPTY, (q_it & 1u) ^ 1u, abort_flag, p);
     if (!ok) break;
-    mbar_arrive_expect_tx(bars + 8 * B_Q_FULL, U.n_active * G::TILE_BYTES);
-    for (int t = 0; t < U.n_active; ++t)
-      for (int c = 0; c < G::NCH; ++c)
-        tma_load_3d(sbase + G::Q_OFF + t * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
-                    bars + 8 * B_Q_FULL, c * G::CW, U.q0 + t * BM, U.bh);
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bars + 8 * B_Q_FULL, U.n_active * G::TILE_BYTES);
+      for (int t = 0; t < U.n_active; ++t)
+        for (int c = 0; c < G::NCH; ++c)
+          tma_load_3d(sbase + G::Q_OFF + t * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
+                      bars + 8 * B_Q_FULL, c * G::CW, U.q0 + t * BM, U.bh);
+    }
+    __syncwarp();
     q_last = q_it & 1;
     ++q_it;
     const int kvz = U.b * p.H_kv + U.g;
@@ -337,19 +347,25 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       const int j = block_at(U, idx);
       const int s = kv_it % NUM_STAGES;
       const uint32_t ph = (kv_it / NUM_STAGES) & 1u;
-      ok = wait_or_abort(bars + 8 * (B_K_EMPTY + s), ph ^ 1u, abort_flag, p);
+      ok = warp_wait(bars + 8 * (B_K_EMPTY + s), ph ^ 1u, abort_flag, p);
       if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (B_K_FULL + s), G::TILE_BYTES);
-      for (int c = 0; c < G::NCH; ++c)
-        tma_load_3d(sbase + G::K_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmK,
-                    bars + 8 * (B_K_FULL + s), c * G::CW, j * BN, kvz);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bars + 8 * (B_K_FULL + s), G::TILE_BYTES);
+        for (int c = 0; c < G::NCH; ++c)
+          tma_load_3d(sbase + G::K_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmK,
+                      bars + 8 * (B_K_FULL + s), c * G::CW, j * BN, kvz);
+      }
+      __syncwarp();
       k_last[s] = ph;
-      ok = wait_or_abort(bars + 8 * (B_V_EMPTY + s), ph ^ 1u, abort_flag, p);
+      ok = warp_wait(bars + 8 * (B_V_EMPTY + s), ph ^ 1u, abort_flag, p);
       if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (B_V_FULL + s), G::TILE_BYTES);
-      for (int c = 0; c < G::NCH; ++c)
-        tma_load_3d(sbase + G::V_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmV,
-                    bars + 8 * (B_V_FULL + s), c * G::CW, j * BN, kvz);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bars + 8 * (B_V_FULL + s), G::TILE_BYTES);
+        for (int c = 0; c < G::NCH; ++c)
+          tma_load_3d(sbase + G::V_OFF + s * G::TILE_BYTES + c * G::CHUNK_BYTES, tmV,
+                      bars + 8 * (B_V_FULL + s), c * G::CW, j * BN, kvz);
+      }
+      __syncwarp();
       v_last[s] = ph;
     }
   }
@@ -410,7 +426,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     const Unit U = decode_unit(u, p);
-    ok = wait_or_abort(bars + 8 * B_Q_FULL, q_ph, abort_flag, p);
+    ok = warp_wait(bars + 8 * B_Q_FULL, q_ph, abort_flag, p);
     if (!ok) break;
     q_ph ^= 1u;
     tc_fence_after_sync();
@@ -418,23 +434,26 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
     {
       const int j0 = block_at(U, 0);
       const int s = kv_it % NUM_STAGES;
-      ok = wait_or_abort(bars + 8 * (B_K_FULL + s), (kv_it / NUM_STAGES) & 1u, abort_flag, p);
+      ok = warp_wait(bars + 8 * (B_K_FULL + s), (kv_it / NUM_STAGES) & 1u, abort_flag, p);
       if (!ok) break;
       tc_fence_after_sync();
-      for (int t = 0; t < 2; ++t)
-        if (tile_uses(U, t, j0)) {
-          issue_qk<D, BF16>(tmem, sbase, t, s);
-          mma_commit(bars + 8 * (B_S_FULL + t));
-        }
-      mma_commit(bars + 8 * (B_K_EMPTY + s));
-      if (U.n_iter == 1) mma_commit(bars + 8 * B_Q_EMPTY);
+      if (elect_one()) {
+        for (int t = 0; t < 2; ++t)
+          if (tile_uses(U, t, j0)) {
+            issue_qk<D, BF16>(tmem, sbase, t, s);
+            mma_commit(bars + 8 * (B_S_FULL + t));
+          }
+        mma_commit(bars + 8 * (B_K_EMPTY + s));
+        if (U.n_iter == 1) mma_commit(bars + 8 * B_Q_EMPTY);
+      }
+      __syncwarp();
     }
     int pv_done[2] = {0, 0};
     for (int idx = 0; idx < U.n_iter && ok; ++idx) {
       const int j = block_at(U, idx);
       const uint32_t it = kv_it + idx;
       const int s = it % NUM_STAGES;
-      ok = wait_or_abort(bars + 8 * (B_V_FULL + s), (it / NUM_STAGES) & 1u, abort_flag, p);
+      ok = warp_wait(bars + 8 * (B_V_FULL + s), (it / NUM_STAGES) & 1u, abort_flag, p);
       if (!ok) break;
       const bool has_next = idx + 1 < U.n_iter;
       const int jn = has_next ? block_at(U, idx + 1) : 0;
@@ -442,47 +461,60 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       const int sn = itn % NUM_STAGES;
       // Q tile 0: P0 V_j, then S0 for the next block
       if (tile_uses(U, 0, j)) {
-        ok = wait_or_abort(bars + 8 * (B_P_FULL + 0), p_ph[0], abort_flag, p);
+        ok = warp_wait(bars + 8 * (B_P_FULL + 0), p_ph[0], abort_flag, p);
         if (!ok) break;
         p_ph[0] ^= 1u;
         tc_fence_after_sync();
-        issue_pv<D, BF16>(tmem, sbase, 0, s, pv_done[0] > 0);
+        if (elect_one()) {
+          issue_pv<D, BF16>(tmem, sbase, 0, s, pv_done[0] > 0);
+          if (j == tile_last_block(U, 0)) mma_commit(bars + 8 * (B_O_FULL + 0));
+        }
+        __syncwarp();
         ++pv_done[0];
-        if (j == tile_last_block(U, 0)) mma_commit(bars + 8 * (B_O_FULL + 0));
       }
       if (has_next) {
-        ok = wait_or_abort(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
+        ok = warp_wait(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
         if (!ok) break;
         tc_fence_after_sync();
         if (tile_uses(U, 0, jn)) {
-          issue_qk<D, BF16>(tmem, sbase, 0, sn);
-          mma_commit(bars + 8 * (B_S_FULL + 0));
+          if (elect_one()) {
+            issue_qk<D, BF16>(tmem, sbase, 0, sn);
+            mma_commit(bars + 8 * (B_S_FULL + 0));
+          }
+          __syncwarp();
         }
       }
       // Q tile 1: P1 V_j, then S1 for the next block
       if (tile_uses(U, 1, j)) {
-        ok = wait_or_abort(bars + 8 * (B_P_FULL + 1), p_ph[1], abort_flag, p);
+        ok = warp_wait(bars + 8 * (B_P_FULL + 1), p_ph[1], abort_flag, p);
         if (!ok) break;
         p_ph[1] ^= 1u;
         tc_fence_after_sync();
-        issue_pv<D, BF16>(tmem, sbase, 1, s, pv_done[1] > 0);
-        ++pv_done[1];
-        if (j == tile_last_block(U, 1)) mma_commit(bars + 8 * (B_O_FULL + 1));
-      }
-      mma_commit(bars + 8 * (B_V_EMPTY + s));
-      if (has_next) {
-        if (tile_uses(U, 1, jn)) {
-          issue_qk<D, BF16>(tmem, sbase, 1, sn);
-          mma_commit(bars + 8 * (B_S_FULL + 1));
+        if (elect_one()) {
+          issue_pv<D, BF16>(tmem, sbase, 1, s, pv_done[1] > 0);
+          if (j == tile_last_block(U, 1)) mma_commit(bars + 8 * (B_O_FULL + 1));
         }
-        mma_commit(bars + 8 * (B_K_EMPTY + sn));
-        if (idx + 2 == U.n_iter) mma_commit(bars + 8 * B_Q_EMPTY);
+        __syncwarp();
+        ++pv_done[1];
       }
+      if (elect_one()) {
+        mma_commit(bars + 8 * (B_V_EMPTY + s));
+        if (has_next) {
+          if (tile_uses(U, 1, jn)) {
+            issue_qk<D, BF16>(tmem, sbase, 1, sn);
+            mma_commit(bars + 8 * (B_S_FULL + 1));
+          }
+          mma_commit(bars + 8 * (B_K_EMPTY + sn));
+          if (idx + 2 == U.n_iter) mma_commit(bars + 8 * B_Q_EMPTY);
+        }
+      }
+      __syncwarp();
     }
     kv_it += U.n_iter;
   }
-  // Every MMA this thread issued has completed once the drain barrier flips.
-  mma_commit(bars + 8 * B_DRAIN);
+  // Every MMA this warp issued has completed once the drain barrier flips.
+  if (elect_one()) mma_commit(bars + 8 * B_DRAIN);
+  __syncwarp();
   drain_wait(bars + 8 * B_DRAIN, 0, p.watchdog_ns);
 }
 
@@ -724,9 +756,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else {
     regs_decrease<CONTROL_REGS>();
     if (warp == MMA_WARP) {
-      if (lane == 0) mma_role<D, BF16>(p, tmem, sbase, bars, abort_flag);
+      mma_role<D, BF16>(p, tmem, sbase, bars, abort_flag);
     } else if (warp == TMA_WARP) {
-      if (lane == 0) tma_role<D>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
+      tma_role<D>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();
