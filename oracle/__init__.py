@@ -4,12 +4,12 @@ TEST INFRASTRUCTURE ONLY: only tests/, __graft_entry__.smoke() and bench.py's
 cpu_baseline / reference legs may import it.  It shares no code with the CUDA
 library.  See oracle/definition.py for the definition and its citations.
 """
-from .definition import (attention, attention_bh, attention_head, attention_weights,
-                        keep_mask, kept_pairs, kv_head_of, scores)
+from .definition import (alibi_bias, alibi_slopes, attention, attention_bh, attention_head,
+                         attention_weights, keep_mask, kept_pairs, kv_head_of, scores)
 from .tiled import tiled_attention, tiled_kv_outer, tiled_q_outer
 
 __all__ = [
-    "attention", "attention_bh", "attention_head", "attention_weights", "keep_mask",
-    "kept_pairs", "kv_head_of", "scores", "tiled_attention", "tiled_kv_outer",
-    "tiled_q_outer",
+    "alibi_bias", "alibi_slopes", "attention", "attention_bh", "attention_head",
+    "attention_weights", "keep_mask", "kept_pairs", "kv_head_of", "scores", "tiled_attention",
+    "tiled_kv_outer", "tiled_q_outer",
 ]

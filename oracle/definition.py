@@ -21,6 +21,9 @@ pages state that the tiled method reaches that definition exactly:
   Step 7 (the naive full-matrix check).
 * "USAAIO Lesson 91", slide 32 (MQA: H query heads share one K/V head; GQA:
   G groups of query heads share one K/V head each).
+* "USAAIO Lesson 91", slides 20-23 (ALiBi position bias): the logit of query i
+  and key j gets -m_h * |i - j| added before the softmax, with one slope per
+  head, m_h = 2^(-h * 8 / H) for h = 1 .. H.
 
 Readings taken where the pages are open:
 
@@ -35,6 +38,9 @@ Readings taken where the pages are open:
 * Query head h reads K/V head h // (H // H_kv).
 * A row with no kept key is an error here (the API never produces one: the
   diagonal is always kept).
+* With ALiBi the bias is added to the scaled logits, scale * q.k - m_h |i - j|
+  (slide 20 writes the scale as 1 / sqrt(d)), before masking; LSE is then the
+  log-sum-exp of the biased logits.
 
 All arithmetic is float64.  Inputs are expected to be the exact float64
 upcast of the 16-bit values the GPU consumes.
@@ -68,6 +74,22 @@ def keep_mask(n_q: int, n_k: int, causal: bool, window: int = 0, n_sink: int = 0
     return keep
 
 
+def alibi_slopes(H: int) -> np.ndarray:
+    """ALiBi slopes of H heads: the geometric sequence m_h = 2^(-h * 8 / H),
+    h = 1 .. H ("USAAIO Lesson 91", slide 23), in float64."""
+    if H < 1:
+        raise ValueError("H must be positive")
+    return np.array([2.0 ** (-h * 8.0 / H) for h in range(1, H + 1)])
+
+
+def alibi_bias(n_k: int, slope: float, rows: np.ndarray) -> np.ndarray:
+    """-slope * |i - j| for query rows ``rows`` and keys 0 .. n_k - 1
+    ("USAAIO Lesson 91", slide 20: logit(i, j) = q_i.k_j / sqrt(d) - m_h |i - j|)."""
+    i = np.asarray(rows, np.float64)[:, None]
+    j = np.arange(n_k, dtype=np.float64)[None, :]
+    return -float(slope) * np.abs(i - j)
+
+
 def scores(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
     """scale * q k^T in float64 (the logits before masking)."""
     return float(scale) * (np.asarray(q, np.float64) @ np.asarray(k, np.float64).T)
@@ -85,11 +107,12 @@ def attention_weights(q, k, scale, causal, window=0, n_sink=0, rows=None):
     return p / p.sum(axis=1, keepdims=True)
 
 
-def attention_head(q, k, v, scale, causal, window=0, n_sink=0, rows=None):
+def attention_head(q, k, v, scale, causal, window=0, n_sink=0, rows=None, slope=0.0):
     """O and LSE for one head.
 
     q: [n_rows, d] (the query rows ``rows`` of the head, or all of them),
-    k, v: [N, d].  Returns (O [n_rows, d], LSE [n_rows]).
+    k, v: [N, d]; ``slope``: the head's ALiBi slope (0 = no bias).
+    Returns (O [n_rows, d], LSE [n_rows]).
     """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -99,6 +122,8 @@ def attention_head(q, k, v, scale, causal, window=0, n_sink=0, rows=None):
         rows = np.arange(q.shape[0])
     rows = np.asarray(rows)
     s = scores(q, k, scale)
+    if slope:
+        s = s + alibi_bias(n, slope, rows)
     keep = keep_mask(n, n, causal, window, n_sink, rows)
     if not keep.any(axis=1).all():
         raise ValueError("a query row has no kept key")
@@ -118,9 +143,10 @@ def kv_head_of(h: int, H: int, H_kv: int) -> int:
     return h // (H // H_kv)
 
 
-def attention(Q, K, V, scale, causal=False, window=0, n_sink=0):
+def attention(Q, K, V, scale, causal=False, window=0, n_sink=0, slopes=None):
     """Full forward for [B, H, N, d] queries and [B, H_kv, N, d] keys/values.
 
+    ``slopes``: optional ALiBi slope per query head ([H]).
     Returns (O [B, H, N, d] float64, LSE [B, H, N] float64).
     """
     Q = np.asarray(Q, np.float64)
@@ -132,12 +158,15 @@ def attention(Q, K, V, scale, causal=False, window=0, n_sink=0):
     L = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
-            O[b, h], L[b, h] = attention_bh(Q, K, V, b, h, scale, causal, window, n_sink)
+            O[b, h], L[b, h] = attention_bh(Q, K, V, b, h, scale, causal, window, n_sink,
+                                            slopes=slopes)
     return O, L
 
 
-def attention_bh(Q, K, V, b, h, scale, causal=False, window=0, n_sink=0, rows=None):
+def attention_bh(Q, K, V, b, h, scale, causal=False, window=0, n_sink=0, rows=None,
+                 slopes=None):
     """O and LSE of head (b, h) for all query rows, or the given ``rows``."""
+    slope = 0.0 if slopes is None else float(slopes[h])
     H, N = Q.shape[1], Q.shape[2]
     g = kv_head_of(h, H, K.shape[1])
     q_all = Q[b, h]
@@ -148,13 +177,13 @@ def attention_bh(Q, K, V, b, h, scale, causal=False, window=0, n_sink=0, rows=No
     rows = np.asarray(rows)
     if rows.size * N <= _MAX_SCORE_ENTRIES:
         return attention_head(np.asarray(q_all[rows], np.float64), k, v, scale,
-                               causal, window, n_sink, rows)
+                              causal, window, n_sink, rows, slope)
     o = np.empty((rows.size, V.shape[3]))
     lse = np.empty(rows.size)
     for c0 in range(0, rows.size, _ROW_CHUNK):
         r = rows[c0:c0 + _ROW_CHUNK]
         o[c0:c0 + r.size], lse[c0:c0 + r.size] = attention_head(
-            np.asarray(q_all[r], np.float64), k, v, scale, causal, window, n_sink, r)
+            np.asarray(q_all[r], np.float64), k, v, scale, causal, window, n_sink, r, slope)
     return o, lse
 
 

@@ -19,6 +19,9 @@ divide N).  One reading is added to the pages' update: when every key seen so
 far in a row is masked, m_new is -inf and exp(m_old - m_new) would be
 exp(-inf + inf) = NaN, so the rescale factor is taken as 0 there (nothing has
 been accumulated yet) and the exponent reference is taken as 0.
+
+With ALiBi ("USAAIO Lesson 91", slides 20-23) each tile's logits get
+-slope * |i - j| added before masking, exactly as in the full matrix.
 """
 from __future__ import annotations
 
@@ -41,7 +44,7 @@ def _block_update(m, l, o, s, v):
     return m_new, l, o
 
 
-def tiled_q_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16):
+def tiled_q_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16, slope=0.0):
     """Q-outer / KV-inner tiled attention of one head; returns (O, LSE)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -60,6 +63,8 @@ def tiled_q_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16):
         for j in range(0, j_end, bs):
             kj, vj = k[j:j + bs], v[j:j + bs]
             s = scale * (qi @ kj.T)
+            if slope:
+                s = s - slope * np.abs(rows[:, None] - np.arange(j, j + kj.shape[0])[None, :])
             keep = keep_mask(n, n, causal, window, n_sink, rows)[:, j:j + kj.shape[0]]
             s = np.where(keep, s, -np.inf)
             m, l, o = _block_update(m, l, o, s, vj)
@@ -68,7 +73,7 @@ def tiled_q_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16):
     return out, lse
 
 
-def tiled_kv_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16):
+def tiled_kv_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16, slope=0.0):
     """KV-outer / Q-inner tiled attention of one head; returns (O, LSE)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -82,13 +87,16 @@ def tiled_kv_outer(q, k, v, scale, causal, window=0, n_sink=0, bs=16):
         for i in range(0, n, bs):
             rows = np.arange(i, min(n, i + bs))
             s = scale * (q[i:i + bs] @ kj.T)
+            if slope:
+                s = s - slope * np.abs(rows[:, None] - np.arange(j, j + kj.shape[0])[None, :])
             keep = keep_mask(n, n, causal, window, n_sink, rows)[:, j:j + kj.shape[0]]
             s = np.where(keep, s, -np.inf)
             m[rows], l[rows], o[rows] = _block_update(m[rows], l[rows], o[rows], s, vj)
     return o / l[:, None], m + np.log(l)
 
 
-def tiled_attention(Q, K, V, scale, causal=False, window=0, n_sink=0, bs=16, order="q"):
+def tiled_attention(Q, K, V, scale, causal=False, window=0, n_sink=0, bs=16, order="q",
+                    slopes=None):
     """Batched wrapper over [B, H, N, d] / [B, H_kv, N, d] inputs."""
     fn = tiled_q_outer if order == "q" else tiled_kv_outer
     B, H, N = Q.shape[:3]
@@ -97,5 +105,7 @@ def tiled_attention(Q, K, V, scale, causal=False, window=0, n_sink=0, bs=16, ord
     for b in range(B):
         for h in range(H):
             g = kv_head_of(h, H, K.shape[1])
-            O[b, h], L[b, h] = fn(Q[b, h], K[b, g], V[b, g], scale, causal, window, n_sink, bs)
+            sl = 0.0 if slopes is None else float(slopes[h])
+            O[b, h], L[b, h] = fn(Q[b, h], K[b, g], V[b, g], scale, causal, window, n_sink, bs,
+                                  sl)
     return O, L
