@@ -5,7 +5,11 @@ One step = one forward (one launch of the attention kernel) over the whole
 workload with inputs resident in HBM.  Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload c3] [--no-cpu-baseline]
+                    [--workload c3] [--no-cpu-baseline] [--alibi]
+
+``--alibi`` times the same workload through attn_fwd_alibi with the pages'
+slopes 2^(-8 h / H) (an extra measurement, not the headline line; it has no
+host-buffer leg and no CPU-oracle leg).
 
 FLOPs are algorithmic: 4 * d * (kept query-key pairs) per head, summed over
 B * H heads (the causal mask keeps N (N + 1) / 2 pairs); masked work is not
@@ -318,6 +322,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--clocks-csv", default=None, help="keep the raw nvidia-smi samples here")
+    ap.add_argument("--alibi", action="store_true",
+                    help="add the ALiBi bias with the pages' slopes (attn_fwd_alibi)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -355,11 +361,12 @@ def main():
     pairs = A.unmasked_pairs(w.N, w.causal, w.window, w.n_sink)
     flops = 4.0 * w.B * w.H * w.d * pairs
     stream = torch.cuda.current_stream(dev)
+    slopes = A.alibi_slopes(w.H, dev) if args.alibi else None
 
     def step(i):
         qd, kd, vd, od, ld = sets[i % n_sets]
         A.attention(qd, kd, vd, causal=w.causal, window=w.window, n_sink=w.n_sink, scale=w.scale,
-                    out=od, lse=ld)
+                    out=od, lse=ld, alibi_slopes=slopes)
 
     def barrier():
         if dist is not None:
@@ -399,24 +406,28 @@ def main():
 
     # ---- end to end through the public host-buffer entry point
     e2e_steps = args.e2e_steps or max(3, min(K, 30))
+    if args.alibi:
+        e2e_steps = 0
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     lh = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
     staging = {"q": sets[0][0], "k": sets[0][1], "v": sets[0][2], "o": sets[0][3], "lse": sets[0][4]}
-    for _ in range(2):
-        A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
-                              window=w.window, n_sink=w.n_sink, scale=w.scale)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
-                              window=w.window, n_sink=w.n_sink, scale=w.scale)
-    e1.record(stream)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
-    e2e_value = whole_job_tflops(world, flops, e2e_steps, e2e_ms)
+    e2e_value = None
+    if e2e_steps:
+        for _ in range(2):
+            A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
+                                  window=w.window, n_sink=w.n_sink, scale=w.scale)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=w.causal,
+                                  window=w.window, n_sink=w.n_sink, scale=w.scale)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+        e2e_value = whole_job_tflops(world, flops, e2e_steps, e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
@@ -424,7 +435,7 @@ def main():
 
     if rank == 0:
         peaks = load_peaks()
-        traffic = load_traffic(w.name)
+        traffic = None if args.alibi else load_traffic(w.name)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -436,7 +447,9 @@ def main():
                        "parallelism": f"replicas x{world} (independent problems, no collective)",
                        "l2": f"inputs larger than L2: {n_sets} rotating device input sets of "
                              f"{per_set_bytes / 2**20:.0f} MiB (L2 126 MiB)",
-                       "flops_per_step": flops, "kept_pairs_per_head": pairs},
+                       "flops_per_step": flops, "kept_pairs_per_head": pairs,
+                       "alibi": ("slopes 2^(-8 h / H), h = 1..H (attn_fwd_alibi)" if args.alibi
+                                 else None)},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                          "traffic": traffic,
@@ -451,7 +464,11 @@ def main():
             "clocks": clocks,
             "device_status": status,
         }
-        if not args.no_cpu_baseline:
+        if args.alibi:
+            line["e2e"] = {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0,
+                           "path": "none: attn_fwd_host has no ALiBi variant"}
+        if not args.no_cpu_baseline and not args.alibi:
             line["cpu_baseline"] = cpu_oracle_throughput(w.name, q, k, v)
         print(json.dumps(line), flush=True)
     if dist is not None:

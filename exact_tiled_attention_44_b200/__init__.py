@@ -17,7 +17,8 @@ import os
 import torch
 
 __all__ = [
-    "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "unmasked_pairs",
+    "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "attn_fwd_alibi_raw",
+    "alibi_slopes", "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
@@ -34,9 +35,9 @@ ATTN_BF16 = 0
 ATTN_FP16 = 1
 ATTN_OUT_F32 = 0x10
 
-EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_error_string", "attn_unmasked_pairs",
-                    "attn_visited_blocks", "attn_get_status", "attn_set_watchdog_ns",
-                    "attn_launch_count")
+EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_slopes",
+                    "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
+                    "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count")
 
 _LIB = None
 
@@ -65,6 +66,10 @@ def load_library():
     lib.attn_fwd.restype = ci
     lib.attn_fwd_host.argtypes = [vp] * 10 + [ci] * 8 + [cf, ci, vp]
     lib.attn_fwd_host.restype = ci
+    lib.attn_fwd_alibi.argtypes = [vp] * 6 + [ci] * 8 + [cf, ci, vp]
+    lib.attn_fwd_alibi.restype = ci
+    lib.attn_alibi_slopes.argtypes = [ci, ctypes.POINTER(ctypes.c_float)]
+    lib.attn_alibi_slopes.restype = ci
     lib.attn_error_string.argtypes = [ci]
     lib.attn_error_string.restype = ctypes.c_char_p
     lib.attn_unmasked_pairs.argtypes = [ci, ci, ci, ci]
@@ -108,6 +113,17 @@ def launch_count() -> int:
     return int(load_library().attn_launch_count())
 
 
+def alibi_slopes(H: int, device=None) -> torch.Tensor:
+    """The library's ALiBi slopes for H heads (attn_alibi_slopes: 2^(-8 h / H),
+    h = 1..H) as a float32 tensor, moved to ``device`` when given."""
+    buf = (ctypes.c_float * max(H, 1))()
+    rc = int(load_library().attn_alibi_slopes(int(H), buf))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_alibi_slopes")
+    t = torch.tensor(list(buf)[:H], dtype=torch.float32)
+    return t if device is None else t.to(device)
+
+
 def default_scale(d: int) -> float:
     """1/sqrt(d) rounded once to float32 (the "HEAD_DIM ** -0.5" of the Hands-On guide)."""
     return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
@@ -128,6 +144,14 @@ def attn_fwd_raw(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scal
                                        n_sink, ctypes.c_float(scale), dtype, stream))
 
 
+def attn_fwd_alibi_raw(q, k, v, o, lse, slopes, B, H, H_kv, N, d, causal, window, n_sink, scale,
+                       dtype, stream) -> int:
+    """Direct C-ABI call of attn_fwd_alibi with integer pointers; returns the status code."""
+    return int(load_library().attn_fwd_alibi(q, k, v, o, lse, slopes, B, H, H_kv, N, d,
+                                             int(causal), window, n_sink, ctypes.c_float(scale),
+                                             dtype, stream))
+
+
 def _check(q, k, v):
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be 4-D [B, H, N, d] / [B, H_kv, N, d]")
@@ -144,10 +168,13 @@ def _check(q, k, v):
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
               window: int = 0, n_sink: int = 0, scale: float | None = None,
               out_f32: bool = False, out: torch.Tensor | None = None,
-              lse: torch.Tensor | None = None, return_lse: bool = True):
+              lse: torch.Tensor | None = None, return_lse: bool = True,
+              alibi_slopes: torch.Tensor | None = None):
     """O = softmax(scale * q k^T + mask) v and the per-row natural-log LSE.
 
     q: [B, H, N, d] CUDA bf16/fp16; k, v: [B, H_kv, N, d] (H % H_kv == 0).
+    ``alibi_slopes``: optional float32 CUDA tensor [H]; the logits then get
+    -slopes[h] * |i - j| added (attn_fwd_alibi).
     Returns (o, lse) with o [B, H, N, d] (float32 when ``out_f32``) and lse
     [B, H, N] float32 (None when ``return_lse`` is False).
     """
@@ -164,12 +191,22 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     stream = torch.cuda.current_stream(q.device).cuda_stream
+    if alibi_slopes is not None:
+        if (alibi_slopes.dtype != torch.float32 or alibi_slopes.device != q.device
+                or tuple(alibi_slopes.shape) != (H,) or not alibi_slopes.is_contiguous()):
+            raise ValueError("alibi_slopes must be a contiguous float32 [H] tensor on q's device")
     with torch.cuda.device(q.device):
-        rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                          lse.data_ptr() if lse is not None else None, B, H, H_kv, N, d, causal,
-                          window, n_sink, scale, code, stream)
+        if alibi_slopes is None:
+            rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else None, B, H, H_kv, N, d,
+                              causal, window, n_sink, scale, code, stream)
+        else:
+            rc = attn_fwd_alibi_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None,
+                                    alibi_slopes.data_ptr(), B, H, H_kv, N, d, causal, window,
+                                    n_sink, scale, code, stream)
     if rc != ATTN_OK:
-        raise AttnError(rc)
+        raise AttnError(rc, "attn_fwd" if alibi_slopes is None else "attn_fwd_alibi")
     return out, lse
 
 

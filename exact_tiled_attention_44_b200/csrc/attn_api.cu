@@ -145,10 +145,10 @@ int encode_map(CUtensorMap* map, const void* base, bool bf16, int d, int n, int 
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool BF16, bool F32>
+template <int D, bool BF16, bool F32, bool ALIBI>
 int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
                const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
-  auto kern = attn::attn_fwd_kernel<D, BF16, F32>;
+  auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI>;
   // At least half of the SM's shared memory, so that two CTAs can never share
   // an SM (each allocates all 512 TMEM columns).
   const int smem_need = attn::Geo<D>::SMEM_BYTES + 1024;
@@ -172,25 +172,29 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+template <int D, bool ALIBI>
+int launch_da(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
+              const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
+  const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
+  const int bit = dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
+  if (bf16)
+    return f32 ? launch_one<D, true, true, ALIBI>(st, bit, mq, mk, mv, kp, stream)
+               : launch_one<D, true, false, ALIBI>(st, bit, mq, mk, mv, kp, stream);
+  return f32 ? launch_one<D, false, true, ALIBI>(st, bit, mq, mk, mv, kp, stream)
+             : launch_one<D, false, false, ALIBI>(st, bit, mq, mk, mv, kp, stream);
+}
+
 template <int D>
 int launch_d(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
              const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
-  const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
-  const int bit = dbit * 4 + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
-  if (bf16)
-    return f32 ? launch_one<D, true, true>(st, bit, mq, mk, mv, kp, stream)
-               : launch_one<D, true, false>(st, bit, mq, mk, mv, kp, stream);
-  return f32 ? launch_one<D, false, true>(st, bit, mq, mk, mv, kp, stream)
-             : launch_one<D, false, false>(st, bit, mq, mk, mv, kp, stream);
+  return kp.alibi != nullptr ? launch_da<D, true>(st, bf16, f32, mq, mk, mv, kp, stream)
+                             : launch_da<D, false>(st, bf16, f32, mq, mk, mv, kp, stream);
 }
 
-}  // namespace
-
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int H_kv, int N, int d, int causal, int window, int n_sink, float scale, int dtype,
-             void* stream) {
+// attn_fwd with an optional slope array (NULL: no position bias).
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+             const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
+             int n_sink, float scale, int dtype, void* stream) {
   Sizes sz;
   bool empty = false;
   int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype, &sz,
@@ -225,6 +229,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   kp.n_qpairs = (N + 2 * attn::BM - 1) / (2 * attn::BM);
   kp.n_kblocks = (N + attn::BN - 1) / attn::BN;
   kp.num_units = B * H * kp.n_qpairs;
+  kp.alibi = slopes;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
@@ -234,6 +239,41 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     case 128: return launch_d<128>(st, bf16, f32, mq, mk, mv, kp, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int H_kv, int N, int d, int causal, int window, int n_sink, float scale, int dtype,
+             void* stream) {
+  return fwd_impl(q, k, v, o, lse, nullptr, B, H, H_kv, N, d, causal, window, n_sink, scale,
+                  dtype, stream);
+}
+
+int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const float* slopes, int B, int H, int H_kv, int N, int d, int causal,
+                   int window, int n_sink, float scale, int dtype, void* stream) {
+  Sizes sz;
+  bool empty = false;
+  const int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                          &sz, &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  if (slopes == nullptr) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(slopes) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  if (overlaps(slopes, static_cast<size_t>(H) * sizeof(float), o, sz.o_bytes) ||
+      (lse != nullptr && overlaps(slopes, static_cast<size_t>(H) * sizeof(float), lse, sz.lse_bytes)))
+    return ATTN_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, slopes, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                  stream);
+}
+
+int attn_alibi_slopes(int H, float* slopes) {
+  if (H < 1 || slopes == nullptr) return ATTN_ERR_INVALID_ARG;
+  for (int h = 1; h <= H; ++h)
+    slopes[h - 1] = static_cast<float>(std::exp2(-8.0 * h / H));
+  return ATTN_OK;
 }
 
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, void* dq,

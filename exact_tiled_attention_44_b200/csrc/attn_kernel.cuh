@@ -22,8 +22,10 @@
 //
 // Per K/V block j and Q tile t:
 //   MMA warp   S_t = Q_t K_j^T         (tcgen05.mma, A and B from smem, fp32 in TMEM)
-//   softmax t  reads S_t row-per-thread (tcgen05.ld 32x32b), masks boundary
-//              blocks, updates m and l, writes P_t = exp2(s*scale*log2e - m)
+//   softmax t  reads S_t row-per-thread (tcgen05.ld 32x32b), adds the ALiBi
+//              bias -slope_h |i - j| when asked ("USAAIO Lesson 91", slides
+//              20-23), masks boundary blocks, updates m and l, writes
+//              P_t = exp2(s*scale*log2e - m)
 //              as 16-bit over the first half of S_t's columns, and rescales
 //              O_t in TMEM when the max grew by more than 2^8 (lazy rescale:
 //              otherwise the stale max is kept; exact, because O and l share it)
@@ -70,6 +72,7 @@ struct KernelParams {
   int n_qpairs;       // ceil(N / 256)
   int n_kblocks;      // ceil(N / 128)
   int num_units;      // B * H * n_qpairs
+  const float* alibi; // ALiBi slope per query head ([H], device), used by the ALIBI kernels
 };
 
 // Shared-memory geometry for head dimension D (16-bit elements).  A 128 x D
@@ -519,7 +522,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   drain_wait(bars + 8 * B_DRAIN, 0, p.watchdog_ns);
 }
 
-template <int D, bool BF16, bool OUT_F32>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI>
 __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars, int t,
                              int warp_in_wg, int lane, volatile int* abort_flag) {
   using G = Geo<D>;
@@ -539,6 +542,9 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
     if (t >= U.n_active) continue;
     const int r0 = U.q0 + t * BM;
     const int row = r0 + row_in_tile;
+    // ALiBi slope of this query head in log2 units (the logits are kept in
+    // units of log2 so that exp2 can be used)
+    const float slope2 = ALIBI ? p.alibi[U.h] * 1.4426950408889634f : 0.f;
     float m_run = -INFINITY, l_exact = 0.f, l_round = 0.f;
     bool first = true;
     for (int idx = 0; idx < U.n_iter; ++idx) {
@@ -553,18 +559,41 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
       const int c0 = j * BN;
       const bool masked = block_needs_mask(p, r0, c0);
       float m_blk;
-      if (masked) {
-        // Scale first, then drop masked keys with -inf (any sign of scale).
-        // Kept keys of this row, in block-local columns e = j - c0:
+      if (masked || ALIBI) {
+        // Scale first (adding the position bias -slope |i - j|), then drop
+        // masked keys with -inf (any sign of scale).  Kept keys of this row,
+        // in block-local columns e = j - c0:
         //   e <= hi (causal limit and key padding) and (e >= lo (window) or e < sk (sinks))
         const int hi = (p.causal ? min(row, p.N - 1) : p.N - 1) - c0;
         const int lo = p.window > 0 ? row - p.window + 1 - c0 : -(1 << 30);
         const int sk = p.window > 0 ? p.n_sink - c0 : -(1 << 30);
+        const float rel = static_cast<float>(row - c0);   // i - c0, exact in fp32
+        if (ALIBI && !masked && p.causal) {
+          // Every key of an unmasked causal block is at or before the row, so
+          // |i - j| = rel - e >= 0: the distance is formed exactly (small
+          // integers), then scaled by the slope once.
+          const float2 rel2 = make_float2(rel, rel);
+          const float2 nsl2 = make_float2(-slope2, -slope2);
+          const float2 c2 = make_float2(c, c);
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const float x = __uint_as_float(sr[e]) * c;
-          const bool keep = (e <= hi) && (e >= lo || e < sk);
-          sr[e] = __float_as_uint(keep ? x : -INFINITY);
+          for (int e = 0; e < 128; e += 2) {
+            const float2 dist = sub2(rel2, make_float2(static_cast<float>(e), static_cast<float>(e + 1)));
+            const float2 s2 = make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            const float2 x = fma2(dist, nsl2, mul2(s2, c2));
+            sr[e] = __float_as_uint(x.x);
+            sr[e + 1] = __float_as_uint(x.y);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            float x = __uint_as_float(sr[e]) * c;
+            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(rel - static_cast<float>(e)), x);
+            if (masked) {
+              const bool keep = (e <= hi) && (e >= lo || e < sk);
+              x = keep ? x : -INFINITY;
+            }
+            sr[e] = __float_as_uint(x);
+          }
         }
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
@@ -604,7 +633,7 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
         m_run = m_new;
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 cc2 = masked ? make_float2(1.f, 1.f) : make_float2(c, c);
+      const float2 cc2 = (masked || ALIBI) ? make_float2(1.f, 1.f) : make_float2(c, c);
       const float2 nm2 = make_float2(-mref, -mref);
       // Two denominators: le sums the fp32 weights (for the LSE), lr sums the
       // same 16-bit-rounded weights the P V MMA consumes (for O, so that every
@@ -697,7 +726,7 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
   }
 }
 
-template <int D, bool BF16, bool OUT_F32>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KernelParams p) {
@@ -751,7 +780,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // smaller one.
   if (warp < 8) {
     regs_increase<SOFTMAX_REGS>();
-    softmax_role<D, BF16, OUT_F32>(p, tmem, bars, warp / 4, warp % 4, lane, abort_flag);
+    softmax_role<D, BF16, OUT_F32, ALIBI>(p, tmem, bars, warp / 4, warp % 4, lane, abort_flag);
     tc_fence_before_sync();
     __syncthreads();
   } else {

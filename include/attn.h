@@ -107,6 +107,34 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
                   int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
                   float scale, int dtype, void* stream);
 
+/*
+ * attn_fwd_alibi -- attn_fwd with the ALiBi position bias ("USAAIO Lesson 91",
+ * slides 20-23, "ALiBi position bias"): the logit of query i and key j is
+ *
+ *     scale * q_i . k_j  -  slopes[h] * |i - j|
+ *
+ * before masking and the softmax, for query head h.  LSE is the log-sum-exp of
+ * these biased, masked logits.  The bias is added for every kept key, causal
+ * or not (|i - j| on both sides of the diagonal).
+ *
+ *   slopes device, [H] float32, one slope per query head, 4-byte aligned, read
+ *          only; any finite values (the pages' choice is attn_alibi_slopes).
+ *          NULL is ATTN_ERR_INVALID_ARG; it must not overlap o or lse.
+ * Every other argument, the layouts, the mask and the errors are those of
+ * attn_fwd.
+ */
+int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const float* slopes, int B, int H, int H_kv, int N, int d, int causal,
+                   int window, int n_sink, float scale, int dtype, void* stream);
+
+/*
+ * attn_alibi_slopes -- host only: writes the pages' ALiBi slopes for H heads,
+ * the geometric sequence slopes[h - 1] = 2^(-8 h / H), h = 1 .. H ("USAAIO
+ * Lesson 91", slide 23), rounded to float32, into the caller's host array
+ * `slopes` of H floats.  Returns ATTN_ERR_INVALID_ARG for H < 1 or NULL.
+ */
+int attn_alibi_slopes(int H, float* slopes);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_error_string(int status);
 

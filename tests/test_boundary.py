@@ -131,3 +131,52 @@ def test_visited_blocks_workloads():
     assert A.visited_blocks(1024, 1) == 36
     assert A.visited_blocks(16384, 1) == 128 * 129 // 2
     assert A.visited_blocks(64, 1) == 1
+
+
+# ------------------------------------------------------------------ ALiBi entry points
+
+
+P_S = 0x600000   # fake, aligned slopes address
+
+
+def call_alibi(slopes=P_S, **kw):
+    a = dict(q=P_Q, k=P_K, v=P_V, o=P_O, lse=P_L, B=1, H=2, H_kv=2, N=100, d=64, causal=1,
+             window=0, n_sink=0, scale=0.125, dtype=A.ATTN_BF16)
+    a.update(kw)
+    return A.attn_fwd_alibi_raw(a["q"], a["k"], a["v"], a["o"], a["lse"], slopes, a["B"], a["H"],
+                                a["H_kv"], a["N"], a["d"], a["causal"], a["window"], a["n_sink"],
+                                a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(slopes=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(slopes=P_S + 2), A.ATTN_ERR_MISALIGNED),
+    (dict(slopes=P_O + 8), A.ATTN_ERR_INVALID_ARG),      # overlaps o
+    (dict(d=48), A.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=0, window=8), A.ATTN_ERR_UNSUPPORTED),
+    (dict(H=6, H_kv=4), A.ATTN_ERR_INVALID_ARG),
+    (dict(q=P_Q + 8), A.ATTN_ERR_MISALIGNED),
+])
+def test_alibi_invalid_calls_are_rejected_before_launch(kw, expect):
+    assert call_alibi(**kw) == expect
+
+
+def test_alibi_empty_problem_is_a_no_op():
+    # nothing to compute: OK before any pointer (slopes included) is looked at
+    assert call_alibi(B=0, slopes=None) == A.ATTN_OK
+    assert call_alibi(N=0) == A.ATTN_OK
+
+
+@pytest.mark.parametrize("H", [1, 2, 4, 8, 12, 16, 32, 64])
+def test_alibi_slopes_helper_matches_pages_formula(H):
+    """attn_alibi_slopes (host) against the oracle's slope sequence, rounded once to fp32."""
+    got = A.alibi_slopes(H)
+    want = torch.tensor(oracle.alibi_slopes(H), dtype=torch.float64).to(torch.float32)
+    assert got.dtype == torch.float32 and torch.equal(got, want)
+
+
+def test_alibi_slopes_helper_rejects_bad_h():
+    lib = A.load_library()
+    buf = (ctypes.c_float * 4)()
+    assert lib.attn_alibi_slopes(0, buf) == A.ATTN_ERR_INVALID_ARG
+    assert lib.attn_alibi_slopes(4, None) == A.ATTN_ERR_INVALID_ARG
