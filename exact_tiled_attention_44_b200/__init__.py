@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "attn_fwd_alibi_raw",
     "alibi_slopes", "unmasked_pairs",
-    "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "error_string",
+    "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
+    "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
     "ATTN_BF16", "ATTN_FP16", "ATTN_OUT_F32",
@@ -37,7 +38,8 @@ ATTN_OUT_F32 = 0x10
 
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_slopes",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
-                    "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count")
+                    "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
+                    "attn_test_withhold_loads")
 
 _LIB = None
 
@@ -82,6 +84,8 @@ def load_library():
     lib.attn_set_watchdog_ns.restype = ctypes.c_ulonglong
     lib.attn_launch_count.argtypes = []
     lib.attn_launch_count.restype = ctypes.c_ulonglong
+    lib.attn_test_withhold_loads.argtypes = [ci]
+    lib.attn_test_withhold_loads.restype = ci
     _LIB = lib
     return lib
 
@@ -111,6 +115,12 @@ def set_watchdog_ns(ns: int) -> int:
 
 def launch_count() -> int:
     return int(load_library().attn_launch_count())
+
+
+def test_withhold_loads(n_launches: int) -> int:
+    """Failure-detection hook: the next n launches issue no copies, so their
+    waits run into the watchdog (see include/attn.h)."""
+    return int(load_library().attn_test_withhold_loads(int(n_launches)))
 
 
 def alibi_slopes(H: int, device=None) -> torch.Tensor:

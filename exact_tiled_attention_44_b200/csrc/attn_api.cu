@@ -33,6 +33,7 @@ DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
 std::atomic<unsigned long long> g_watchdog_ns{2000000000ull};
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<int> g_withhold{0};     // launches left that withhold their loads (test hook)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -230,6 +231,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
   kp.n_kblocks = (N + attn::BN - 1) / attn::BN;
   kp.num_units = B * H * kp.n_qpairs;
   kp.alibi = slopes;
+  kp.withhold_loads = 0;
+  for (int n = g_withhold.load(); n > 0;) {
+    if (g_withhold.compare_exchange_weak(n, n - 1)) {
+      kp.withhold_loads = 1;
+      break;
+    }
+  }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
@@ -378,6 +386,12 @@ unsigned long long attn_set_watchdog_ns(unsigned long long ns) {
   if (ns < 1000000ull) ns = 1000000ull;
   if (ns > 60000000000ull) ns = 60000000000ull;
   return g_watchdog_ns.exchange(ns);
+}
+
+int attn_test_withhold_loads(int n_launches) {
+  if (n_launches < 0) return ATTN_ERR_INVALID_ARG;
+  g_withhold.store(n_launches);
+  return ATTN_OK;
 }
 
 unsigned long long attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -73,6 +73,7 @@ struct KernelParams {
   int n_kblocks;      // ceil(N / 128)
   int num_units;      // B * H * n_qpairs
   const float* alibi; // ALiBi slope per query head ([H], device), used by the ALIBI kernels
+  int withhold_loads; // test hook: the TMA warp issues nothing, so every wait runs out
 };
 
 // Shared-memory geometry for head dimension D (16-bit elements).  A 128 x D
@@ -324,6 +325,9 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
                          const CUtensorMap* tmV, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
   using G = Geo<D>;
+  // Failure-detection test: no copy is issued, so the other roles' bounded
+  // waits expire and the CTA reports ATTN_ERR_DEVICE_TIMEOUT and exits.
+  if (p.withhold_loads) return;
   uint32_t q_it = 0, kv_it = 0;
   // parity of the last load issued into each barrier, for the drain
   int q_last = -1, k_last[NUM_STAGES], v_last[NUM_STAGES];

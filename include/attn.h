@@ -173,6 +173,17 @@ unsigned long long attn_set_watchdog_ns(unsigned long long ns);
  * points).  Lets a caller count the GPU launches of a region. */
 unsigned long long attn_launch_count(void);
 
+/*
+ * attn_test_withhold_loads -- failure-detection test hook (the paper has no
+ * counterpart).  The next `n_launches` launches of this process start their
+ * copy warp without issuing a single copy, so every other wait in the kernel
+ * runs into the watchdog: the CTAs record ATTN_ERR_DEVICE_TIMEOUT (read it with
+ * attn_get_status), release their tensor memory and return; outputs are left
+ * unspecified.  Nothing faults and the context stays usable.  0 turns the hook
+ * off.  Returns ATTN_ERR_INVALID_ARG for n_launches < 0.
+ */
+int attn_test_withhold_loads(int n_launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -180,3 +180,8 @@ def test_alibi_slopes_helper_rejects_bad_h():
     buf = (ctypes.c_float * 4)()
     assert lib.attn_alibi_slopes(0, buf) == A.ATTN_ERR_INVALID_ARG
     assert lib.attn_alibi_slopes(4, None) == A.ATTN_ERR_INVALID_ARG
+
+
+def test_withhold_hook_arguments():
+    assert A.test_withhold_loads(-1) == A.ATTN_ERR_INVALID_ARG
+    assert A.test_withhold_loads(0) == A.ATTN_OK
