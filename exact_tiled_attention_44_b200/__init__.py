@@ -18,7 +18,7 @@ import torch
 
 __all__ = [
     "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "attn_fwd_alibi_raw",
-    "alibi_slopes", "unmasked_pairs",
+    "alibi_slopes", "decode", "decode_workspace_bytes", "attn_decode_raw", "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
     "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
@@ -37,6 +37,7 @@ ATTN_FP16 = 1
 ATTN_OUT_F32 = 0x10
 
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_slopes",
+                    "attn_decode", "attn_decode_workspace_bytes",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
                     "attn_test_withhold_loads")
@@ -72,6 +73,10 @@ def load_library():
     lib.attn_fwd_alibi.restype = ci
     lib.attn_alibi_slopes.argtypes = [ci, ctypes.POINTER(ctypes.c_float)]
     lib.attn_alibi_slopes.restype = ci
+    lib.attn_decode.argtypes = [vp] * 6 + [ctypes.c_longlong] + [ci] * 9 + [cf, ci, vp]
+    lib.attn_decode.restype = ci
+    lib.attn_decode_workspace_bytes.argtypes = [ci] * 6
+    lib.attn_decode_workspace_bytes.restype = ctypes.c_longlong
     lib.attn_error_string.argtypes = [ci]
     lib.attn_error_string.restype = ctypes.c_char_p
     lib.attn_unmasked_pairs.argtypes = [ci, ci, ci, ci]
@@ -160,6 +165,63 @@ def attn_fwd_alibi_raw(q, k, v, o, lse, slopes, B, H, H_kv, N, d, causal, window
     return int(load_library().attn_fwd_alibi(q, k, v, o, lse, slopes, B, H, H_kv, N, d,
                                              int(causal), window, n_sink, ctypes.c_float(scale),
                                              dtype, stream))
+
+
+def decode_workspace_bytes(B: int, H: int, H_kv: int, N_q: int, N_kv: int, d: int) -> int:
+    """Scratch bytes attn_decode needs for these sizes (0: the cache is not split)."""
+    return int(load_library().attn_decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d))
+
+
+def attn_decode_raw(q, k, v, o, lse, ws, ws_bytes, B, H, H_kv, N_q, N_kv, d, causal, window,
+                    n_sink, scale, dtype, stream) -> int:
+    """Direct C-ABI call of attn_decode with integer pointers; returns the status code."""
+    return int(load_library().attn_decode(q, k, v, o, lse, ws, ctypes.c_longlong(ws_bytes), B, H,
+                                          H_kv, N_q, N_kv, d, int(causal), window, n_sink,
+                                          ctypes.c_float(scale), dtype, stream))
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = True,
+           window: int = 0, n_sink: int = 0, scale: float | None = None, out_f32: bool = False,
+           out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+           return_lse: bool = True, workspace: torch.Tensor | None = None):
+    """Attention of the new query rows q [B, H, N_q, d] against the cache k, v
+    [B, H_kv, N_kv, d] (attn_decode).  Query row i sits at cache position
+    N_kv - N_q + i.  ``workspace``: a CUDA uint8 tensor of at least
+    decode_workspace_bytes(...) bytes; allocated here (torch) when omitted.
+    Returns (o [B, H, N_q, d], lse [B, H, N_q] or None)."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q [B, H, N_q, d] and k, v [B, H_kv, N_kv, d] expected")
+    if q.shape[0] != k.shape[0] or q.shape[3] != k.shape[3]:
+        raise ValueError(f"shape mismatch q={tuple(q.shape)} k={tuple(k.shape)}")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if not q.is_cuda:
+        raise ValueError("decode() takes CUDA tensors")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    B, H, N_q, d = q.shape
+    H_kv, N_kv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = default_scale(d)
+    code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
+    if out is None:
+        out = torch.empty((B, H, N_q, d), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        rc = attn_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr() if lse is not None else None, ws_ptr, ws_bytes, B, H,
+                             H_kv, N_q, N_kv, d, causal, window, n_sink, scale, code, stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_decode")
+    return out, lse
 
 
 def _check(q, k, v):

@@ -135,6 +135,42 @@ int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* 
  */
 int attn_alibi_slopes(int H, float* slopes);
 
+/*
+ * attn_decode -- attention of N_q new query rows against a K/V cache of N_kv
+ * positions, split across the cache ("USAAIO Lesson 91", slide 31: every
+ * decoding step re-reads the whole cache; slide 32: query heads share K/V
+ * heads; "Building a FlashAttention-style tiled self-attention block in pure
+ * NumPy", "Extending It", item 6: split the sequence, then reduce the partial
+ * outputs).
+ *
+ *   q      device, [B, H, N_q, d] bf16/fp16; query row i sits at cache
+ *          position N_kv - N_q + i (the last N_q tokens of the sequence)
+ *   k, v   device, [B, H_kv, N_kv, d] (the cache), same element type
+ *   o      device, [B, H, N_q, d] (16-bit or float32 with ATTN_OUT_F32)
+ *   lse    device, [B, H, N_q] float32, or NULL
+ *   workspace, workspace_bytes   device scratch of at least
+ *          attn_decode_workspace_bytes(...) bytes, 256-byte aligned, owned by
+ *          the caller and not read by it; may be NULL when that size is 0.
+ *          Its counters are cleared by the call (one cudaMemsetAsync on
+ *          `stream`) and it must not be shared by calls in flight at once.
+ *   1 <= N_q <= N_kv; d is 64 or 128; (H / H_kv) * N_q <= 64 query rows per
+ *          K/V head (else ATTN_ERR_UNSUPPORTED)
+ * The mask rule, scale, dtype, LSE and error conventions are those of
+ * attn_fwd, with the query position N_kv - N_q + i in place of i.  The cache
+ * range is cut into splits of whole 64-key tiles; each split's partial
+ * (O_s, LSE_s) goes to the workspace and the last split of each (b, kv head)
+ * to finish merges them in split order (LSE = ln sum exp(LSE_s),
+ * O = sum exp(LSE_s - LSE) O_s), so results are deterministic.
+ */
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                void* workspace, long long workspace_bytes, int B, int H, int H_kv, int N_q,
+                int N_kv, int d, int causal, int window, int n_sink, float scale, int dtype,
+                void* stream);
+
+/* Host only: bytes of workspace attn_decode needs for these sizes (0 when the
+ * cache is not split), or -1 for invalid sizes.  Independent of the device. */
+long long attn_decode_workspace_bytes(int B, int H, int H_kv, int N_q, int N_kv, int d);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_error_string(int status);
 

@@ -185,3 +185,52 @@ def test_alibi_slopes_helper_rejects_bad_h():
 def test_withhold_hook_arguments():
     assert A.test_withhold_loads(-1) == A.ATTN_ERR_INVALID_ARG
     assert A.test_withhold_loads(0) == A.ATTN_OK
+
+
+# ------------------------------------------------------------------ decode entry points
+
+
+# fake, aligned, never dereferenced addresses far enough apart for a cache of several MB
+D_Q, D_K, D_V, D_O, D_L, D_W = (i << 28 for i in range(1, 7))
+
+
+def call_decode(ws=D_W, ws_bytes=1 << 26, **kw):
+    a = dict(q=D_Q, k=D_K, v=D_V, o=D_O, lse=D_L, B=1, H=8, H_kv=2, N_q=1, N_kv=4096, d=128,
+             causal=1, window=0, n_sink=0, scale=0.088, dtype=A.ATTN_BF16)
+    a.update(kw)
+    return A.attn_decode_raw(a["q"], a["k"], a["v"], a["o"], a["lse"], ws, ws_bytes, a["B"], a["H"],
+                             a["H_kv"], a["N_q"], a["N_kv"], a["d"], a["causal"], a["window"],
+                             a["n_sink"], a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(N_q=5, N_kv=4), A.ATTN_ERR_INVALID_ARG),
+    (dict(d=32), A.ATTN_ERR_UNSUPPORTED),
+    (dict(H=64, H_kv=1, N_q=2), A.ATTN_ERR_UNSUPPORTED),      # 128 rows per K/V head
+    (dict(causal=0, window=8), A.ATTN_ERR_UNSUPPORTED),
+    (dict(H=6, H_kv=4), A.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), A.ATTN_ERR_INVALID_ARG),                  # the cache is split: workspace needed
+    (dict(ws_bytes=16), A.ATTN_ERR_INVALID_ARG),
+    (dict(ws=D_W + 16), A.ATTN_ERR_MISALIGNED),
+    (dict(q=D_Q + 4), A.ATTN_ERR_MISALIGNED),
+    (dict(o=D_K + 64), A.ATTN_ERR_INVALID_ARG),               # o overlaps the cache
+    (dict(ws=D_O), A.ATTN_ERR_INVALID_ARG),                   # workspace overlaps o
+    (dict(ws_bytes=-1), A.ATTN_ERR_INVALID_ARG),
+])
+def test_decode_invalid_calls_are_rejected_before_launch(kw, expect):
+    assert call_decode(**kw) == expect
+
+
+def test_decode_empty_problem_is_a_no_op():
+    assert call_decode(B=0, ws=None, ws_bytes=0) == A.ATTN_OK
+    assert call_decode(N_q=0, ws=None, ws_bytes=0) == A.ATTN_OK
+
+
+def test_decode_workspace_size():
+    # one split (short cache): no workspace
+    assert A.decode_workspace_bytes(4, 8, 2, 1, 200, 128) == 0
+    # split cache: counters, partial LSE and partial O for every split and row
+    b = A.decode_workspace_bytes(1, 8, 2, 1, 4096, 128)
+    assert b >= 8 * 1 * (128 + 1) * 4 * 2
+    assert A.decode_workspace_bytes(1, 8, 2, 5, 4, 128) == -1
+    assert A.decode_workspace_bytes(0, 8, 2, 1, 4096, 128) == 0
