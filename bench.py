@@ -7,6 +7,10 @@ workload with inputs resident in HBM.  Prints ONE JSON line on rank 0.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
                     [--workload c3] [--no-cpu-baseline] [--alibi]
 
+``--decode`` times one decoding step (attn_decode, dec1: B=8 H=32 H_kv=8, one
+new row against an 8192-position cache, d=128 bf16) and reports GB/s of
+algorithmic bytes against the measured HBM bandwidth (an extra line).
+
 ``--alibi`` times the same workload through attn_fwd_alibi with the pages'
 slopes 2^(-8 h / H) (an extra measurement, not the headline line; it has no
 host-buffer leg and no CPU-oracle leg).
@@ -312,6 +316,79 @@ def whole_job_tflops(world: int, flops_per_step: float, steps: int, ms: float) -
 
 # ----------------------------------------------------------------- GPU arm
 
+def decode_bench(args):
+    """--decode: one decoding step per timed step, inputs resident in HBM and
+    rotating over two sets (each larger than L2)."""
+    import torch
+    import exact_tiled_attention_44_b200 as A
+    from exact_tiled_attention_44_b200.inputs import DECODE_WORKLOADS, make_decode_inputs
+
+    w = DECODE_WORKLOADS["dec1"]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    B, H, H_kv, N_q, N_kv, d = w["B"], w["H"], w["H_kv"], w["N_q"], w["N_kv"], w["d"]
+    q, k, v = make_decode_inputs(B, H, H_kv, N_q, N_kv, d)
+    sets = []
+    for i in range(2):
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        sets.append((qd, kd, vd, torch.empty_like(qd), torch.empty(q.shape[:3], device=dev),
+                     torch.empty(A.decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d),
+                                 dtype=torch.uint8, device=dev)))
+    alg_bytes = 2 * (q.numel() * 2) + 2 * k.numel() * 2 + B * H * N_q * 4   # q, o, k, v, lse
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        qd, kd, vd, od, ld, ws = sets[i % 2]
+        A.decode(qd, kd, vd, causal=w["causal"], out=od, lse=ld, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0, args.clocks_csv)
+    sampler.start()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    n0 = A.launch_count()
+    sampler.mark_begin()
+    t0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    launches = A.launch_count() - n0
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    peaks = load_peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    line = {
+        "metric": "attn decode GB/s & % of measured HBM bandwidth (split-KV, one step)",
+        "value": alg_bytes * K / (total_ms / 1e3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+        "config": {"workload": f"dec1: B={B} H={H} H_kv={H_kv} N_q={N_q} N_kv={N_kv} d={d} "
+                               f"{w['dtype']} causal={int(w['causal'])}",
+                   "l2": "inputs larger than L2: 2 rotating sets of "
+                         f"{(q.numel() + 2 * k.numel()) * 2 / 2**20:.0f} MiB (L2 126 MiB)",
+                   "alg_bytes_per_step": alg_bytes,
+                   "splits": A.decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d) > 0},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peaks['source']} HBM copy (MEASURED_PEAKS.json)",
+                     "kernel_ms": kern_ms},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "device_status": A.get_status(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -322,6 +399,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--clocks-csv", default=None, help="keep the raw nvidia-smi samples here")
+    ap.add_argument("--decode", action="store_true",
+                    help="time attn_decode on the dec1 workload (GB/s against HBM)")
     ap.add_argument("--alibi", action="store_true",
                     help="add the ALiBi bias with the pages' slopes (attn_fwd_alibi)")
     args = ap.parse_args()
@@ -329,6 +408,8 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args)
+    if args.decode:
+        return decode_bench(args)
 
     import torch
     import exact_tiled_attention_44_b200 as A

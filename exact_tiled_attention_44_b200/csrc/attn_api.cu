@@ -254,7 +254,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
 // ------------------------------------------------------------ decode
 
 // Split rule (device independent, so that the workspace size can be queried
-// without a device): about two CTAs per SM of a 148-SM part in total, each
+// without a device): at most two CTAs per SM of a 148-SM part in total (one
+// wave; rounding the split count up would leave a short second wave), each
 // split at least 256 keys long and a whole number of 64-key tiles.
 struct DecodePlan {
   int n_splits, split_keys;
@@ -266,7 +267,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 DecodePlan decode_plan(int B, int H, int H_kv, int N_q, int N_kv, int d) {
   DecodePlan pl{};
   const long long groups = static_cast<long long>(B) * H_kv;
-  const long long want = (296 + groups - 1) / groups;
+  const long long want = groups < 296 ? 296 / groups : 1;
   const long long max_splits = (static_cast<long long>(N_kv) + 255) / 256;
   long long s = want < max_splits ? want : max_splits;
   if (s < 1) s = 1;
@@ -335,12 +336,12 @@ int encode_cache_map(CUtensorMap* map, const void* base, bool bf16, int d, int n
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool BF16, bool F32>
-int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
-                  const CUtensorMap& mv, cudaStream_t stream) {
-  auto kern = attn::attn_decode_kernel<D, BF16, F32>;
+template <int D, bool BF16, bool F32, int RW>
+int launch_decode_rw(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
+                     const CUtensorMap& mv, cudaStream_t stream) {
+  auto kern = attn::attn_decode_kernel<D, BF16, F32, RW>;
   const int smem = attn::DecGeo<D>::SMEM_BYTES + 1024;
-  const int bit = (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
+  const int bit = (RW == 1 ? 0 : RW == 4 ? 8 : 16) + (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!(st->dec_attr_set & (1u << bit))) {
@@ -353,6 +354,16 @@ int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorM
   kern<<<grid, attn::DEC_THREADS, smem, stream>>>(mk, mv, dp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Row capacity per warp from the group's query rows G * N_q (4 warps).
+template <int D, bool BF16, bool F32>
+int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
+                  const CUtensorMap& mv, cudaStream_t stream) {
+  const int rows = (dp.H / dp.H_kv) * dp.N_q;
+  if (rows <= attn::DEC_WARPS) return launch_decode_rw<D, BF16, F32, 1>(st, dp, mk, mv, stream);
+  if (rows <= 4 * attn::DEC_WARPS) return launch_decode_rw<D, BF16, F32, 4>(st, dp, mk, mv, stream);
+  return launch_decode_rw<D, BF16, F32, 16>(st, dp, mk, mv, stream);
 }
 
 // attn_decode with an explicit workspace (base + size in bytes).

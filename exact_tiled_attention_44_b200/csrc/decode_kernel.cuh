@@ -35,7 +35,8 @@ constexpr int DEC_T = 64;            // keys per K/V tile
 constexpr int DEC_WARPS = 4;
 constexpr int DEC_THREADS = 32 * DEC_WARPS;
 constexpr int DEC_MAX_ROWS = 64;     // query rows of one (b, g): G * N_q
-constexpr int DEC_ROWS_PER_WARP = DEC_MAX_ROWS / DEC_WARPS;
+// Row capacity per warp is a template parameter RW (1, 4 or 16) chosen from
+// G * N_q, so that small groups do not carry the register arrays of large ones.
 
 struct DecodeParams {
   const void* q;
@@ -110,7 +111,7 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-template <int D, bool BF16, bool OUT_F32>
+template <int D, bool BF16, bool OUT_F32, int RW>
 __global__ void __launch_bounds__(DEC_THREADS, 1)
 attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const DecodeParams p) {
@@ -187,9 +188,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 
   // per-row state of this warp's rows r = warp + 4 rr
   const int nr = (R > warp) ? (R - warp + DEC_WARPS - 1) / DEC_WARPS : 0;
-  float m[DEC_ROWS_PER_WARP], l[DEC_ROWS_PER_WARP], acc[DEC_ROWS_PER_WARP][CPL];
+  float m[RW], l[RW], acc[RW][CPL];
 #pragma unroll
-  for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) {
+  for (int rr = 0; rr < RW; ++rr) {
     m[rr] = -INFINITY;
     l[rr] = 0.f;
 #pragma unroll
@@ -215,9 +216,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     const int j_end = min(j0 + DEC_T, hi);
 
     // S for keys j0 + lane and j0 + 32 + lane, every row of this warp
-    float s0[DEC_ROWS_PER_WARP], s1[DEC_ROWS_PER_WARP];
+    float s0[RW], s1[RW];
 #pragma unroll
-    for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) s0[rr] = s1[rr] = 0.f;
+    for (int rr = 0; rr < RW; ++rr) s0[rr] = s1[rr] = 0.f;
 #pragma unroll 2
     for (int c8 = 0; c8 < D / 8; ++c8) {
       const uint32_t box = static_cast<uint32_t>((c8 / 8) * G::BOX_BYTES);
@@ -236,7 +237,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         fb[2 * u] = y.x; fb[2 * u + 1] = y.y;
       }
 #pragma unroll
-      for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) {
+      for (int rr = 0; rr < RW; ++rr) {
         if (rr < nr) {
           const float4* qr = reinterpret_cast<const float4*>(qs + (warp + DEC_WARPS * rr) * D + c8 * 8);
           const float4 q0 = qr[0], q1 = qr[1];
@@ -252,10 +253,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     }
 
     // mask, online softmax (log2 units, lazy rescale), probabilities
-    float pa[DEC_ROWS_PER_WARP], pb[DEC_ROWS_PER_WARP];
+    float pa[RW], pb[RW];
     const int ja = j0 + lane, jb = j0 + 32 + lane;
 #pragma unroll
-    for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) {
+    for (int rr = 0; rr < RW; ++rr) {
       pa[rr] = pb[rr] = 0.f;
       if (rr < nr) {
         const int r = warp + DEC_WARPS * rr;
@@ -299,7 +300,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         vf[0] = x.x; vf[1] = x.y;
       }
 #pragma unroll
-      for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) {
+      for (int rr = 0; rr < RW; ++rr) {
         if (rr < nr) {
           const float pt = __shfl_sync(0xffffffffu, t < 32 ? pa[rr] : pb[rr], t & 31);
 #pragma unroll
@@ -325,7 +326,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 
   // ---- this split's result for each row of the warp
 #pragma unroll
-  for (int rr = 0; rr < DEC_ROWS_PER_WARP; ++rr) {
+  for (int rr = 0; rr < RW; ++rr) {
     if (rr < nr) {
       const int r = warp + DEC_WARPS * rr;
       const int h = g * G_heads + r / p.N_q, i = r % p.N_q;

@@ -111,6 +111,25 @@ def random_qkv(B, H, H_kv, N, d, dtype=torch.bfloat16, seed=0, std=1.0):
     return tuple(torch.from_numpy(a).to(dtype).contiguous() for a in (q, k, v))
 
 
+# Decode workload: new query rows against a K/V cache (one decoding step of a
+# GQA model; shapes in the range of the pages' KV-cache discussion, "USAAIO
+# Lesson 91", slides 31 and 51).
+DECODE_WORKLOADS = {
+    "dec1": dict(B=8, H=32, H_kv=8, N_q=1, N_kv=8192, d=128, dtype="bf16", causal=True),
+}
+
+
+def make_decode_inputs(B, H, H_kv, N_q, N_kv, d, dtype=torch.bfloat16, seed=0):
+    """q [B, H, N_q, d] and the cache k, v [B, H_kv, N_kv, d]: one
+    numpy.random.default_rng(seed) draws float32 standard normals for q, k, v in
+    that order, rounded to ``dtype``."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, N_q, d), dtype=np.float32)
+    k = rng.standard_normal((B, H_kv, N_kv, d), dtype=np.float32)
+    v = rng.standard_normal((B, H_kv, N_kv, d), dtype=np.float32)
+    return tuple(torch.from_numpy(a).to(dtype).contiguous() for a in (q, k, v))
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact float64 upcast of a 16-bit tensor (every bf16/fp16 value is a float64 value)."""
     return t.detach().to("cpu", torch.float64).numpy()
