@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "attn_fwd_alibi_raw",
-    "alibi_slopes", "decode", "decode_workspace_bytes", "attn_decode_raw", "unmasked_pairs",
+    "alibi_slopes", "decode", "decode_workspace_bytes", "attn_decode_raw",
+    "attn_decode_noalloc_raw", "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
     "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
@@ -37,7 +38,7 @@ ATTN_FP16 = 1
 ATTN_OUT_F32 = 0x10
 
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_slopes",
-                    "attn_decode", "attn_decode_workspace_bytes",
+                    "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
                     "attn_test_withhold_loads")
@@ -77,6 +78,8 @@ def load_library():
     lib.attn_decode.restype = ci
     lib.attn_decode_workspace_bytes.argtypes = [ci] * 6
     lib.attn_decode_workspace_bytes.restype = ctypes.c_longlong
+    lib.attn_decode_noalloc.argtypes = [vp] * 5 + [ci] * 9 + [cf, ci, vp]
+    lib.attn_decode_noalloc.restype = ci
     lib.attn_error_string.argtypes = [ci]
     lib.attn_error_string.restype = ctypes.c_char_p
     lib.attn_unmasked_pairs.argtypes = [ci, ci, ci, ci]
@@ -178,6 +181,14 @@ def attn_decode_raw(q, k, v, o, lse, ws, ws_bytes, B, H, H_kv, N_q, N_kv, d, cau
     return int(load_library().attn_decode(q, k, v, o, lse, ws, ctypes.c_longlong(ws_bytes), B, H,
                                           H_kv, N_q, N_kv, d, int(causal), window, n_sink,
                                           ctypes.c_float(scale), dtype, stream))
+
+
+def attn_decode_noalloc_raw(q, k, v, o, lse, B, H, H_kv, N_q, N_kv, d, causal, window, n_sink,
+                            scale, dtype, stream) -> int:
+    """Direct C-ABI call of attn_decode_noalloc (static scratch); returns the status code."""
+    return int(load_library().attn_decode_noalloc(q, k, v, o, lse, B, H, H_kv, N_q, N_kv, d,
+                                                  int(causal), window, n_sink,
+                                                  ctypes.c_float(scale), dtype, stream))
 
 
 def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = True,

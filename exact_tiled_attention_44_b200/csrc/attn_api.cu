@@ -366,6 +366,29 @@ int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorM
   return launch_decode_rw<D, BF16, F32, 16>(st, dp, mk, mv, stream);
 }
 
+// Static decode scratch for attn_decode_noalloc: part of the module image on
+// every device, so that entry point allocates nothing.  Its address is looked
+// up once per device.
+constexpr size_t kDecodeScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+int decode_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess) return ATTN_ERR_CUDA;
+    g_scratch_addr[dev] = addr;
+  }
+  *out = g_scratch_addr[dev];
+  return ATTN_OK;
+}
+
 // attn_decode with an explicit workspace (base + size in bytes).
 int decode_impl(const void* q, const void* k, const void* v, void* o, float* lse, void* ws,
                 size_t ws_bytes, int B, int H, int H_kv, int N_q, int N_kv, int d, int causal,
@@ -437,6 +460,21 @@ long long attn_decode_workspace_bytes(int B, int H, int H_kv, int N_q, int N_kv,
   if (B < 0 || H < 0 || H_kv < 1 || N_q < 0 || N_kv < 0 || d <= 0 || N_q > N_kv) return -1;
   if (B == 0 || H == 0 || N_q == 0) return 0;
   return static_cast<long long>(decode_plan(B, H, H_kv, N_q, N_kv, d).bytes);
+}
+
+int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int H_kv, int N_q, int N_kv, int d, int causal, int window,
+                        int n_sink, float scale, int dtype, void* stream) {
+  bool empty = false;
+  int rc = validate_decode(q, k, v, o, lse, B, H, H_kv, N_q, N_kv, d, causal, window, n_sink,
+                           scale, dtype, &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  if (decode_plan(B, H, H_kv, N_q, N_kv, d).bytes > kDecodeScratchBytes) return ATTN_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  rc = decode_scratch(&scratch);
+  if (rc != ATTN_OK) return rc;
+  return decode_impl(q, k, v, o, lse, scratch, kDecodeScratchBytes, B, H, H_kv, N_q, N_kv, d,
+                     causal, window, n_sink, scale, dtype, stream);
 }
 
 int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,

@@ -171,6 +171,22 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
  * cache is not split), or -1 for invalid sizes.  Independent of the device. */
 long long attn_decode_workspace_bytes(int B, int H, int H_kv, int N_q, int N_kv, int d);
 
+/*
+ * attn_decode_noalloc -- attn_decode without a caller workspace (the paper has
+ * no counterpart).  The partial results and split counters live in a static
+ * 4 MiB device array that is part of the library image on every device, so
+ * the call allocates nothing; its split counters are cleared on every call
+ * (one cudaMemsetAsync on `stream`).  Sizes whose attn_decode_workspace_bytes
+ * exceed 4 MiB return ATTN_ERR_UNSUPPORTED before anything is enqueued.
+ * Races: every call on a device shares that one array, so calls on one device
+ * must not overlap in time (issue them on one stream, or synchronise the
+ * streams in between); overlapping calls give unspecified results.  All other
+ * arguments and conventions are those of attn_decode.
+ */
+int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int H_kv, int N_q, int N_kv, int d, int causal,
+                        int window, int n_sink, float scale, int dtype, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_error_string(int status);
 
