@@ -29,6 +29,7 @@ struct DeviceState {
   int* status = nullptr;           // device address of g_device_status
   uint32_t attr_set = 0;           // one bit per forward kernel instantiation
   uint32_t dec_attr_set = 0;       // one bit per decode kernel instantiation
+  uint32_t dec_small_attr_set = 0; // one bit per small-group decode kernel instantiation
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -356,13 +357,34 @@ int launch_decode_rw(DeviceState* st, const attn::DecodeParams& dp, const CUtens
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// Row capacity per warp from the group's query rows G * N_q (4 warps).
+template <int D, bool BF16, bool F32, int RMAX>
+int launch_decode_small(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
+                        const CUtensorMap& mv, cudaStream_t stream) {
+  auto kern = attn::attn_decode_small_kernel<D, BF16, F32, RMAX>;
+  const int smem = attn::DecSmallGeo<D, RMAX>::SMEM_BYTES + 1024;
+  const int bit = (RMAX == 4 ? 0 : 8) + (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!(st->dec_small_attr_set & (1u << bit))) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      st->dec_small_attr_set |= 1u << bit;
+    }
+  }
+  const dim3 grid(dp.n_splits, dp.B * dp.H_kv);
+  kern<<<grid, attn::DEC_THREADS, smem, stream>>>(mk, mv, dp);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Kernel by the group's query rows G * N_q: up to 4 and up to 16 rows use the
+// warp-sliced kernel, larger groups (up to 64) the row-per-warp kernel.
 template <int D, bool BF16, bool F32>
 int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
                   const CUtensorMap& mv, cudaStream_t stream) {
   const int rows = (dp.H / dp.H_kv) * dp.N_q;
-  if (rows <= attn::DEC_WARPS) return launch_decode_rw<D, BF16, F32, 1>(st, dp, mk, mv, stream);
-  if (rows <= 4 * attn::DEC_WARPS) return launch_decode_rw<D, BF16, F32, 4>(st, dp, mk, mv, stream);
+  if (rows <= 4) return launch_decode_small<D, BF16, F32, 4>(st, dp, mk, mv, stream);
+  if (rows <= 16) return launch_decode_small<D, BF16, F32, 16>(st, dp, mk, mv, stream);
   return launch_decode_rw<D, BF16, F32, 16>(st, dp, mk, mv, stream);
 }
 

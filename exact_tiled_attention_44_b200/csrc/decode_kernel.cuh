@@ -403,4 +403,379 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   if (threadIdx.x == 0) p.counters[bg] = 0;
 }
 
+
+// ------------------------------------------------------------ small groups
+//
+// Groups of at most 16 query rows (typical decoding: one or a few new tokens,
+// GQA groups up to 16) use a leaner kernel.  Each warp takes its own 16-key
+// slice of every 64-key tile for all rows of the group and keeps its own
+// running (m, l, O): the four warps are four sub-splits of the split, merged
+// once at its end, so every K/V element is converted once and no per-tile
+// exchange between warps is needed.  Lane (key k = lane % 16, row parity
+// lane / 16) forms the dot products of its key with its rows (four partial
+// sums each, to keep the dependency chains short); the probabilities go
+// through shared memory to the P V loop, where each lane owns D / 32 output
+// columns of every row.  Three pipeline stages.
+
+constexpr int DEC_SMALL_STAGES = 3;
+
+template <int D, int RMAX>
+struct DecSmallGeo {
+  static_assert(D == 64 || D == 128, "decode supports d = 64 and 128");
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX_BYTES = DEC_T * 128;
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
+  static constexpr int K_OFF = 0;                                   // stages, then reused for the merge
+  static constexpr int V_OFF = K_OFF + DEC_SMALL_STAGES * TILE_BYTES;
+  static constexpr int Q_OFF = V_OFF + DEC_SMALL_STAGES * TILE_BYTES;   // fp32 [RMAX][D]
+  static constexpr int P_OFF = Q_OFF + RMAX * D * 4;                // fp32 [warp][RMAX][16]
+  static constexpr int A_OFF = P_OFF + DEC_WARPS * RMAX * 16 * 4;   // fp32 [warp][RMAX] rescale
+  static constexpr int BAR_OFF = A_OFF + DEC_WARPS * RMAX * 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + 8 * 2 * DEC_SMALL_STAGES + 16;
+  // end-of-split merge buffers, over the K stages: m, l [warp][RMAX], O [warp][RMAX][D]
+  static constexpr int MM_OFF = K_OFF;
+  static constexpr int ML_OFF = MM_OFF + DEC_WARPS * RMAX * 4;
+  static constexpr int MO_OFF = ML_OFF + DEC_WARPS * RMAX * 4;
+  static_assert(MO_OFF + DEC_WARPS * RMAX * D * 4 <= V_OFF, "merge buffers fit the K stages");
+};
+
+template <int D, bool BF16, bool OUT_F32, int RMAX>
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+  using G = DecSmallGeo<D, RMAX>;
+  constexpr int CPL = D / 32;          // output columns per lane
+  constexpr int RH = RMAX / 2;         // rows per lane in the S phase
+  constexpr int NS = DEC_SMALL_STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bars = sbase + G::BAR_OFF;          // FULL[NS], EMPTY[NS]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + G::BAR_OFF + 8 * 2 * NS);
+  volatile int* last_flag = abort_flag + 1;
+  float* qs = reinterpret_cast<float*>(smem + G::Q_OFF);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int kl = lane & 15, hf = lane >> 4;
+  const int split = blockIdx.x, bg = blockIdx.y;
+  const int b = bg / p.H_kv, g = bg % p.H_kv;
+  const int G_heads = p.H / p.H_kv;
+  const int R = G_heads * p.N_q;
+  const int lo = split * p.split_keys, hi = min(p.N_kv, lo + p.split_keys);
+  float* ps = reinterpret_cast<float*>(smem + G::P_OFF) + warp * RMAX * 16;
+  float* as = reinterpret_cast<float*>(smem + G::A_OFF) + warp * RMAX;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bars + 8 * s, 1);
+      mbar_init(bars + 8 * (NS + s), DEC_WARPS);
+    }
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  for (int e = threadIdx.x; e < RMAX * (D / 2); e += DEC_THREADS) {
+    const int r = e / (D / 2), c2 = e % (D / 2);
+    float2 f = make_float2(0.f, 0.f);
+    if (r < R) {
+      const int h = g * G_heads + r / p.N_q, i = r % p.N_q;
+      const size_t off = ((static_cast<size_t>(b) * p.H + h) * p.N_q + i) * D + 2 * c2;
+      f = unpack2f<BF16>(*reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.q) + off));
+    }
+    qs[r * D + 2 * c2] = f.x * p.scale_log2;
+    qs[r * D + 2 * c2 + 1] = f.y * p.scale_log2;
+  }
+  __syncthreads();
+
+  const int j_first = dec_next_tile(p, lo, hi);
+  bool ok = true;
+  int issued_last[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) issued_last[s] = -1;
+  auto issue = [&](int j0, int n) {
+    const int st = n % NS;
+    const uint32_t ph = static_cast<uint32_t>(n / NS) & 1u;
+    const uint32_t empty = bars + 8 * (NS + st);
+    if (!mbar_try_wait(empty, ph ^ 1u) &&
+        !wait_slow(empty, ph ^ 1u, abort_flag, p.status, p.watchdog_ns))
+      return false;
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bars + 8 * st, 2 * G::TILE_BYTES);
+      for (int c = 0; c < G::NBOX; ++c) {
+        tma_load_3d(sbase + G::K_OFF + st * G::TILE_BYTES + c * G::BOX_BYTES, &tmK, bars + 8 * st,
+                    c * 64, j0, bg);
+        tma_load_3d(sbase + G::V_OFF + st * G::TILE_BYTES + c * G::BOX_BYTES, &tmV, bars + 8 * st,
+                    c * 64, j0, bg);
+      }
+    }
+    __syncwarp();
+    issued_last[st] = static_cast<int>(ph);
+    return true;
+  };
+  // prologue: the first NS - 1 tiles
+  int j_pre = j_first;
+  if (warp == 0) {
+    for (int n = 0; n < NS - 1 && j_pre < hi && ok; ++n) {
+      ok = __all_sync(0xffffffffu, issue(j_pre, n));
+      j_pre = dec_next_tile(p, j_pre + DEC_T, hi);
+    }
+  }
+
+  float m[RH], l[RH], acc[RMAX][CPL];
+#pragma unroll
+  for (int rr = 0; rr < RH; ++rr) {
+    m[rr] = -INFINITY;
+    l[rr] = 0.f;
+  }
+#pragma unroll
+  for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[r][c] = 0.f;
+
+  int n = 0;
+  for (int j0 = j_first; j0 < hi && ok; j0 = dec_next_tile(p, j0 + DEC_T, hi), ++n) {
+    const int st = n % NS;
+    if (warp == 0) {
+      if (j_pre < hi) {
+        ok = __all_sync(0xffffffffu, issue(j_pre, n + NS - 1));
+        j_pre = dec_next_tile(p, j_pre + DEC_T, hi);
+      }
+      if (!ok) break;
+    }
+    {
+      const uint32_t full = bars + 8 * st, ph = static_cast<uint32_t>(n / NS) & 1u;
+      ok = __all_sync(0xffffffffu, mbar_try_wait(full, ph) ||
+                                       wait_slow(full, ph, abort_flag, p.status, p.watchdog_ns));
+    }
+    if (!ok) break;
+    const uint32_t ks = sbase + G::K_OFF + st * G::TILE_BYTES;
+    const uint32_t vs = sbase + G::V_OFF + st * G::TILE_BYTES;
+    const int t = warp * 16 + kl;                  // this lane's key within the tile
+    const int j = j0 + t;
+
+    // S for key j and rows r = hf + 2 rr, four partial sums each
+    float sa[RH][4];
+#pragma unroll
+    for (int rr = 0; rr < RH; ++rr)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) sa[rr][u] = 0.f;
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      uint32_t kw[4];
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(kw[0]), "=r"(kw[1]), "=r"(kw[2]), "=r"(kw[3])
+                   : "r"(ks + (c8 / 8) * G::BOX_BYTES + sw128(t, c8 % 8)));
+      float kf[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 x = unpack2f<BF16>(kw[u]);
+        kf[2 * u] = x.x;
+        kf[2 * u + 1] = x.y;
+      }
+#pragma unroll
+      for (int rr = 0; rr < RH; ++rr) {
+        const int r = hf + 2 * rr;
+        if (r < R) {
+          const float4* qr = reinterpret_cast<const float4*>(qs + r * D + c8 * 8);
+          const float4 q0 = qr[0], q1 = qr[1];
+          sa[rr][0] = fmaf(q0.x, kf[0], sa[rr][0]);
+          sa[rr][1] = fmaf(q0.y, kf[1], sa[rr][1]);
+          sa[rr][2] = fmaf(q0.z, kf[2], sa[rr][2]);
+          sa[rr][3] = fmaf(q0.w, kf[3], sa[rr][3]);
+          sa[rr][0] = fmaf(q1.x, kf[4], sa[rr][0]);
+          sa[rr][1] = fmaf(q1.y, kf[5], sa[rr][1]);
+          sa[rr][2] = fmaf(q1.z, kf[6], sa[rr][2]);
+          sa[rr][3] = fmaf(q1.w, kf[7], sa[rr][3]);
+        }
+      }
+    }
+
+    // masking and online softmax over this warp's 16 keys (one half-warp per
+    // row parity); P and the rescale factors go to shared memory
+    const int j_end = min(j0 + DEC_T, hi);
+#pragma unroll
+    for (int rr = 0; rr < RH; ++rr) {
+      const int r = hf + 2 * rr;                   // rows >= R carry -inf and stay inert
+      const int pos = p.N_kv - p.N_q + r % p.N_q;
+      const bool keep = r < R && j < j_end && (!p.causal || j <= pos) &&
+                        (p.window == 0 || pos - j < p.window || j < p.n_sink);
+      const float x = keep ? (sa[rr][0] + sa[rr][1]) + (sa[rr][2] + sa[rr][3]) : -INFINITY;
+      // row max over the 16 keys of this half-warp (all 32 lanes shuffle)
+      float bmax = x;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+      float alpha = 1.f;
+      const float m_new = fmaxf(m[rr], bmax);
+      if (m_new > m[rr] + RESCALE_THRESHOLD) {
+        alpha = (m[rr] == -INFINITY) ? 0.f : fast_exp2(m[rr] - m_new);
+        l[rr] *= alpha;
+        m[rr] = m_new;
+      }
+      const float pj = fast_exp2(x - ((m[rr] == -INFINITY) ? 0.f : m[rr]));
+      l[rr] += pj;
+      ps[r * 16 + kl] = pj;
+      if (kl == 0) as[r] = alpha;
+    }
+    __syncwarp();
+
+    // O += P V over this warp's 16 keys; lane owns columns CPL * lane ..
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+      if (r < R) {
+        const float a = as[r];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[r][c] *= a;
+      }
+    }
+#pragma unroll
+    for (int k4 = 0; k4 < 16; k4 += 4) {
+      float vf[4][CPL];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int tv = warp * 16 + k4 + kk;
+        if constexpr (D == 128) {
+          uint32_t w0, w1;
+          const uint32_t a = vs + (lane / 16) * G::BOX_BYTES + sw128(tv, (lane % 16) / 2) + (lane & 1) * 8;
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a));
+          const float2 x = unpack2f<BF16>(w0), y = unpack2f<BF16>(w1);
+          vf[kk][0] = x.x; vf[kk][1] = x.y; vf[kk][2] = y.x; vf[kk][3] = y.y;
+        } else {
+          uint32_t w0;
+          const uint32_t a = vs + sw128(tv, lane / 4) + (lane & 3) * 4;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(a));
+          const float2 x = unpack2f<BF16>(w0);
+          vf[kk][0] = x.x; vf[kk][1] = x.y;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RMAX; ++r) {
+        if (r < R) {
+          const float4 p4 = *reinterpret_cast<const float4*>(ps + r * 16 + k4);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            float o = acc[r][c];
+            o = fmaf(p4.x, vf[0][c], o);
+            o = fmaf(p4.y, vf[1][c], o);
+            o = fmaf(p4.z, vf[2][c], o);
+            o = fmaf(p4.w, vf[3][c], o);
+            acc[r][c] = o;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + 8 * (NS + st));
+  }
+
+  if (!__syncthreads_and(ok ? 1 : 0)) {
+    if (warp == 0) {
+      for (int s = 0; s < NS; ++s)
+        if (issued_last[s] >= 0) drain_wait(bars + 8 * s, issued_last[s], p.watchdog_ns);
+    }
+    return;
+  }
+
+  // ---- merge the four warps' sub-splits (buffers over the now idle K stages)
+  float* mm = reinterpret_cast<float*>(smem + G::MM_OFF);
+  float* ml = reinterpret_cast<float*>(smem + G::ML_OFF);
+  float* mo = reinterpret_cast<float*>(smem + G::MO_OFF);
+#pragma unroll
+  for (int rr = 0; rr < RH; ++rr) {
+    const int r = hf + 2 * rr;
+    float lt = l[rr];
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+    if (r < RMAX && kl == 0) {
+      mm[warp * RMAX + r] = (r < R) ? m[rr] : -INFINITY;
+      ml[warp * RMAX + r] = (r < R) ? lt : 0.f;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) mo[(warp * RMAX + r) * D + CPL * lane + c] = acc[r][c];
+  __syncthreads();
+
+  const size_t split_stride = static_cast<size_t>(p.B) * p.H * p.N_q;
+  for (int e = threadIdx.x; e < R * D; e += DEC_THREADS) {
+    const int r = e / D, c = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, mm[w * RMAX + r]);
+    float lt = 0.f, o = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < DEC_WARPS; ++w) {
+        const float mw = mm[w * RMAX + r];
+        if (mw == -INFINITY) continue;
+        const float s = fast_exp2(mw - M);
+        lt = fmaf(s, ml[w * RMAX + r], lt);
+        o = fmaf(s, mo[(w * RMAX + r) * D + c], o);
+      }
+    }
+    const bool has = lt > 0.f;
+    const float ov = has ? o / lt : 0.f;
+    const float lse_nat = has ? (M + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+    const int h = g * G_heads + r / p.N_q, i = r % p.N_q;
+    const size_t row_idx = (static_cast<size_t>(b) * p.H + h) * p.N_q + i;
+    if (p.n_splits == 1) {
+      if constexpr (OUT_F32) {
+        static_cast<float*>(p.o)[row_idx * D + c] = ov;
+      } else if constexpr (BF16) {
+        static_cast<__nv_bfloat16*>(p.o)[row_idx * D + c] = __float2bfloat16_rn(ov);
+      } else {
+        static_cast<__half*>(p.o)[row_idx * D + c] = __float2half_rn(ov);
+      }
+      if (c == 0 && p.lse != nullptr) p.lse[row_idx] = lse_nat;
+    } else {
+      const size_t ws_row = static_cast<size_t>(split) * split_stride + row_idx;
+      p.ws_o[ws_row * D + c] = ov;
+      if (c == 0) p.ws_lse[ws_row] = lse_nat;
+    }
+  }
+  if (p.n_splits == 1) return;
+
+  // ---- the last split of this (b, g) to finish merges all of them
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(p.counters + bg, 1);
+    *last_flag = (prev == p.n_splits - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < R * D; e += DEC_THREADS) {
+    const int r = e / D, c = e % D;
+    const int h = g * G_heads + r / p.N_q, i = r % p.N_q;
+    const size_t row_idx = (static_cast<size_t>(b) * p.H + h) * p.N_q + i;
+    float mx = -INFINITY;
+    for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, __ldcg(p.ws_lse + s * split_stride + row_idx));
+    float tot = 0.f;
+    for (int s = 0; s < p.n_splits; ++s) {
+      const float ls = __ldcg(p.ws_lse + s * split_stride + row_idx);
+      tot += (ls == -INFINITY) ? 0.f : __expf(ls - mx);
+    }
+    const float lse_nat = mx + __logf(tot);
+    float o = 0.f;
+    for (int s = 0; s < p.n_splits; ++s) {
+      const float ls = __ldcg(p.ws_lse + s * split_stride + row_idx);
+      if (ls == -INFINITY) continue;
+      o = fmaf(__expf(ls - lse_nat), __ldcg(p.ws_o + (s * split_stride + row_idx) * D + c), o);
+    }
+    if constexpr (OUT_F32) {
+      static_cast<float*>(p.o)[row_idx * D + c] = o;
+    } else if constexpr (BF16) {
+      static_cast<__nv_bfloat16*>(p.o)[row_idx * D + c] = __float2bfloat16_rn(o);
+    } else {
+      static_cast<__half*>(p.o)[row_idx * D + c] = __float2half_rn(o);
+    }
+    if (c == 0 && p.lse != nullptr) p.lse[row_idx] = lse_nat;
+  }
+  if (threadIdx.x == 0) p.counters[bg] = 0;
+}
+
 }  // namespace attn
