@@ -357,11 +357,11 @@ int launch_decode_rw(DeviceState* st, const attn::DecodeParams& dp, const CUtens
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool BF16, bool F32, int RMAX>
+template <int D, bool BF16, bool F32, int RMAX, int NW>
 int launch_decode_small(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
                         const CUtensorMap& mv, cudaStream_t stream) {
-  auto kern = attn::attn_decode_small_kernel<D, BF16, F32, RMAX>;
-  const int smem = attn::DecSmallGeo<D, RMAX>::SMEM_BYTES + 1024;
+  auto kern = attn::attn_decode_small_kernel<D, BF16, F32, RMAX, NW>;
+  const int smem = attn::DecSmallGeo<D, RMAX, NW>::SMEM_BYTES + 1024;
   const int bit = (RMAX == 4 ? 0 : 8) + (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -372,7 +372,7 @@ int launch_decode_small(DeviceState* st, const attn::DecodeParams& dp, const CUt
     }
   }
   const dim3 grid(dp.n_splits, dp.B * dp.H_kv);
-  kern<<<grid, attn::DEC_THREADS, smem, stream>>>(mk, mv, dp);
+  kern<<<grid, NW * 32, smem, stream>>>(mk, mv, dp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -383,8 +383,8 @@ template <int D, bool BF16, bool F32>
 int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
                   const CUtensorMap& mv, cudaStream_t stream) {
   const int rows = (dp.H / dp.H_kv) * dp.N_q;
-  if (rows <= 4) return launch_decode_small<D, BF16, F32, 4>(st, dp, mk, mv, stream);
-  if (rows <= 16) return launch_decode_small<D, BF16, F32, 16>(st, dp, mk, mv, stream);
+  if (rows <= 4) return launch_decode_small<D, BF16, F32, 4, 8>(st, dp, mk, mv, stream);
+  if (rows <= 16) return launch_decode_small<D, BF16, F32, 16, 4>(st, dp, mk, mv, stream);
   return launch_decode_rw<D, BF16, F32, 16>(st, dp, mk, mv, stream);
 }
 

@@ -407,19 +407,20 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 // ------------------------------------------------------------ small groups
 //
 // Groups of at most 16 query rows (typical decoding: one or a few new tokens,
-// GQA groups up to 16) use a leaner kernel.  Each warp takes its own 16-key
-// slice of every 64-key tile for all rows of the group and keeps its own
-// running (m, l, O): the four warps are four sub-splits of the split, merged
-// once at its end, so every K/V element is converted once and no per-tile
-// exchange between warps is needed.  Lane (key k = lane % 16, row parity
-// lane / 16) forms the dot products of its key with its rows (four partial
-// sums each, to keep the dependency chains short); the probabilities go
-// through shared memory to the P V loop, where each lane owns D / 32 output
-// columns of every row.  Three pipeline stages.
+// GQA groups up to 16) use a leaner kernel.  Each of the NW warps takes its
+// own slice of KPW = 64 / NW keys of every 64-key tile for all rows of the
+// group and keeps its own running (m, l, O): the warps are sub-splits of the
+// split, merged once at its end, so every K/V element is converted once and
+// no per-tile exchange between warps is needed.  Lane (key lane % KPW, row
+// group lane / KPW) forms the dot products of its key with its rows (four
+// partial sums each, to keep the dependency chains short); the probabilities
+// go through shared memory to the P V loop, where each lane owns D / 32
+// output columns of every row.  Three pipeline stages.  More warps per CTA
+// (NW = 8 for groups of up to 4 rows) hide more latency per scheduler.
 
 constexpr int DEC_SMALL_STAGES = 3;
 
-template <int D, int RMAX>
+template <int D, int RMAX, int NW>
 struct DecSmallGeo {
   static_assert(D == 64 || D == 128, "decode supports d = 64 and 128");
   static constexpr int NBOX = D / 64;
@@ -428,24 +429,30 @@ struct DecSmallGeo {
   static constexpr int K_OFF = 0;                                   // stages, then reused for the merge
   static constexpr int V_OFF = K_OFF + DEC_SMALL_STAGES * TILE_BYTES;
   static constexpr int Q_OFF = V_OFF + DEC_SMALL_STAGES * TILE_BYTES;   // fp32 [RMAX][D]
-  static constexpr int P_OFF = Q_OFF + RMAX * D * 4;                // fp32 [warp][RMAX][16]
-  static constexpr int A_OFF = P_OFF + DEC_WARPS * RMAX * 16 * 4;   // fp32 [warp][RMAX] rescale
-  static constexpr int BAR_OFF = A_OFF + DEC_WARPS * RMAX * 4;
+  static constexpr int KPW = DEC_T / NW;                           // keys per warp per tile
+  static constexpr int P_OFF = Q_OFF + RMAX * D * 4;                // fp32 [warp][RMAX][KPW]
+  static constexpr int A_OFF = P_OFF + NW * RMAX * KPW * 4;         // fp32 [warp][RMAX] rescale
+  static constexpr int BAR_OFF = A_OFF + NW * RMAX * 4;
   static constexpr int SMEM_BYTES = BAR_OFF + 8 * 2 * DEC_SMALL_STAGES + 16;
   // end-of-split merge buffers, over the K stages: m, l [warp][RMAX], O [warp][RMAX][D]
   static constexpr int MM_OFF = K_OFF;
-  static constexpr int ML_OFF = MM_OFF + DEC_WARPS * RMAX * 4;
-  static constexpr int MO_OFF = ML_OFF + DEC_WARPS * RMAX * 4;
-  static_assert(MO_OFF + DEC_WARPS * RMAX * D * 4 <= V_OFF, "merge buffers fit the K stages");
+  static constexpr int ML_OFF = MM_OFF + NW * RMAX * 4;
+  static constexpr int MO_OFF = ML_OFF + NW * RMAX * 4;
+  static_assert(MO_OFF + NW * RMAX * D * 4 <= V_OFF, "merge buffers fit the K stages");
+  static_assert(KPW % 4 == 0 && 32 % KPW == 0, "key slice per warp");
 };
 
-template <int D, bool BF16, bool OUT_F32, int RMAX>
-__global__ void __launch_bounds__(DEC_THREADS, 1)
+template <int D, bool BF16, bool OUT_F32, int RMAX, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
 attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-  using G = DecSmallGeo<D, RMAX>;
+  using G = DecSmallGeo<D, RMAX, NW>;
+  constexpr int NT = NW * 32;
+  constexpr int KPW = G::KPW;
+  constexpr int RQ = 32 / KPW;         // row groups per warp in the S phase
   constexpr int CPL = D / 32;          // output columns per lane
-  constexpr int RH = RMAX / 2;         // rows per lane in the S phase
+  constexpr int RH = RMAX / RQ;        // rows per lane in the S phase
+  static_assert(RH >= 1, "row capacity");
   constexpr int NS = DEC_SMALL_STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -457,19 +464,19 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
   float* qs = reinterpret_cast<float*>(smem + G::Q_OFF);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int kl = lane & 15, hf = lane >> 4;
+  const int kl = lane % KPW, hf = lane / KPW;
   const int split = blockIdx.x, bg = blockIdx.y;
   const int b = bg / p.H_kv, g = bg % p.H_kv;
   const int G_heads = p.H / p.H_kv;
   const int R = G_heads * p.N_q;
   const int lo = split * p.split_keys, hi = min(p.N_kv, lo + p.split_keys);
-  float* ps = reinterpret_cast<float*>(smem + G::P_OFF) + warp * RMAX * 16;
+  float* ps = reinterpret_cast<float*>(smem + G::P_OFF) + warp * RMAX * KPW;
   float* as = reinterpret_cast<float*>(smem + G::A_OFF) + warp * RMAX;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(bars + 8 * s, 1);
-      mbar_init(bars + 8 * (NS + s), DEC_WARPS);
+      mbar_init(bars + 8 * (NS + s), NW);
     }
     *abort_flag = 0;
     *last_flag = 0;
@@ -477,7 +484,7 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  for (int e = threadIdx.x; e < RMAX * (D / 2); e += DEC_THREADS) {
+  for (int e = threadIdx.x; e < RMAX * (D / 2); e += NT) {
     const int r = e / (D / 2), c2 = e % (D / 2);
     float2 f = make_float2(0.f, 0.f);
     if (r < R) {
@@ -553,10 +560,10 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
     if (!ok) break;
     const uint32_t ks = sbase + G::K_OFF + st * G::TILE_BYTES;
     const uint32_t vs = sbase + G::V_OFF + st * G::TILE_BYTES;
-    const int t = warp * 16 + kl;                  // this lane's key within the tile
+    const int t = warp * KPW + kl;                 // this lane's key within the tile
     const int j = j0 + t;
 
-    // S for key j and rows r = hf + 2 rr, four partial sums each
+    // S for key j and rows r = hf + RQ rr, four partial sums each
     float sa[RH][4];
 #pragma unroll
     for (int rr = 0; rr < RH; ++rr)
@@ -577,7 +584,7 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
       }
 #pragma unroll
       for (int rr = 0; rr < RH; ++rr) {
-        const int r = hf + 2 * rr;
+        const int r = hf + RQ * rr;
         if (r < R) {
           const float4* qr = reinterpret_cast<const float4*>(qs + r * D + c8 * 8);
           const float4 q0 = qr[0], q1 = qr[1];
@@ -593,20 +600,20 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
       }
     }
 
-    // masking and online softmax over this warp's 16 keys (one half-warp per
-    // row parity); P and the rescale factors go to shared memory
+    // masking and online softmax over this warp's KPW keys (one lane group per
+    // row group); P and the rescale factors go to shared memory
     const int j_end = min(j0 + DEC_T, hi);
 #pragma unroll
     for (int rr = 0; rr < RH; ++rr) {
-      const int r = hf + 2 * rr;                   // rows >= R carry -inf and stay inert
+      const int r = hf + RQ * rr;                  // rows >= R carry -inf and stay inert
       const int pos = p.N_kv - p.N_q + r % p.N_q;
       const bool keep = r < R && j < j_end && (!p.causal || j <= pos) &&
                         (p.window == 0 || pos - j < p.window || j < p.n_sink);
       const float x = keep ? (sa[rr][0] + sa[rr][1]) + (sa[rr][2] + sa[rr][3]) : -INFINITY;
-      // row max over the 16 keys of this half-warp (all 32 lanes shuffle)
+      // row max over the KPW keys of this lane group (all 32 lanes shuffle)
       float bmax = x;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+      for (int o = KPW / 2; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
       float alpha = 1.f;
       const float m_new = fmaxf(m[rr], bmax);
       if (m_new > m[rr] + RESCALE_THRESHOLD) {
@@ -616,12 +623,12 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
       }
       const float pj = fast_exp2(x - ((m[rr] == -INFINITY) ? 0.f : m[rr]));
       l[rr] += pj;
-      ps[r * 16 + kl] = pj;
+      ps[r * KPW + kl] = pj;
       if (kl == 0) as[r] = alpha;
     }
     __syncwarp();
 
-    // O += P V over this warp's 16 keys; lane owns columns CPL * lane ..
+    // O += P V over this warp's KPW keys; lane owns columns CPL * lane ..
 #pragma unroll
     for (int r = 0; r < RMAX; ++r) {
       if (r < R) {
@@ -631,11 +638,11 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
       }
     }
 #pragma unroll
-    for (int k4 = 0; k4 < 16; k4 += 4) {
+    for (int k4 = 0; k4 < KPW; k4 += 4) {
       float vf[4][CPL];
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const int tv = warp * 16 + k4 + kk;
+        const int tv = warp * KPW + k4 + kk;
         if constexpr (D == 128) {
           uint32_t w0, w1;
           const uint32_t a = vs + (lane / 16) * G::BOX_BYTES + sw128(tv, (lane % 16) / 2) + (lane & 1) * 8;
@@ -653,7 +660,7 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
       for (int r = 0; r < RMAX; ++r) {
         if (r < R) {
-          const float4 p4 = *reinterpret_cast<const float4*>(ps + r * 16 + k4);
+          const float4 p4 = *reinterpret_cast<const float4*>(ps + r * KPW + k4);
 #pragma unroll
           for (int c = 0; c < CPL; ++c) {
             float o = acc[r][c];
@@ -684,10 +691,10 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
   float* mo = reinterpret_cast<float*>(smem + G::MO_OFF);
 #pragma unroll
   for (int rr = 0; rr < RH; ++rr) {
-    const int r = hf + 2 * rr;
+    const int r = hf + RQ * rr;
     float lt = l[rr];
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+    for (int o = KPW / 2; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
     if (r < RMAX && kl == 0) {
       mm[warp * RMAX + r] = (r < R) ? m[rr] : -INFINITY;
       ml[warp * RMAX + r] = (r < R) ? lt : 0.f;
@@ -700,15 +707,15 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
   __syncthreads();
 
   const size_t split_stride = static_cast<size_t>(p.B) * p.H * p.N_q;
-  for (int e = threadIdx.x; e < R * D; e += DEC_THREADS) {
+  for (int e = threadIdx.x; e < R * D; e += NT) {
     const int r = e / D, c = e % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, mm[w * RMAX + r]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mm[w * RMAX + r]);
     float lt = 0.f, o = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < DEC_WARPS; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float mw = mm[w * RMAX + r];
         if (mw == -INFINITY) continue;
         const float s = fast_exp2(mw - M);
@@ -748,7 +755,7 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
   __syncthreads();
   if (!*last_flag) return;
   __threadfence();
-  for (int e = threadIdx.x; e < R * D; e += DEC_THREADS) {
+  for (int e = threadIdx.x; e < R * D; e += NT) {
     const int r = e / D, c = e % D;
     const int h = g * G_heads + r / p.N_q, i = r % p.N_q;
     const size_t row_idx = (static_cast<size_t>(b) * p.H + h) * p.N_q + i;
