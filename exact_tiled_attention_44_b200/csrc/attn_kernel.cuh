@@ -44,6 +44,7 @@ namespace attn {
 constexpr int BM = 128;           // query rows per Q tile
 constexpr int BN = 128;           // keys per K/V block
 constexpr int NUM_STAGES = 2;     // K ring depth (and V ring depth)
+constexpr int Q_SLOTS = 3;        // Q tile slots
 constexpr int NUM_THREADS = 384;           // three warpgroups
 constexpr int MMA_WARP = 8;
 constexpr int TMA_WARP = 9;
@@ -88,8 +89,11 @@ struct Geo {
   static constexpr int CHUNK_BYTES = 128 * CB;
   // descriptor layout field: 6 = 32B swizzle, 4 = 64B, 2 = 128B
   static constexpr uint32_t LAYOUT = CB == 128 ? 2u : (CB == 64 ? 4u : 6u);
+  // Three Q tile slots rotate over the CTA's units (tile t of the CTA's u-th
+  // unit uses slot (2u + t) % 3), so the next unit's tile 0 lands in a slot
+  // that is free long before the current unit ends.
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
+  static constexpr int K_OFF = Q_OFF + Q_SLOTS * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + NUM_STAGES * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + NUM_STAGES * TILE_BYTES;
   static constexpr int SMEM_BYTES = BAR_OFF + 256;
@@ -97,12 +101,13 @@ struct Geo {
   static constexpr uint32_t O_COL0 = 256;    // O_t at column 256 + D t
   static_assert(D % 16 == 0 && D <= 128, "unsupported head dim");
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory budget");
 };
 
 // Barrier slots (8 bytes each) after the tiles.
 enum BarSlot : int {
-  B_Q_FULL = 0, B_Q_EMPTY = 1,
-  B_K_FULL = 2, B_K_EMPTY = B_K_FULL + NUM_STAGES,
+  B_Q_FULL = 0, B_Q_EMPTY = B_Q_FULL + Q_SLOTS,   // [Q_SLOTS] each
+  B_K_FULL = B_Q_EMPTY + Q_SLOTS, B_K_EMPTY = B_K_FULL + NUM_STAGES,
   B_V_FULL = B_K_EMPTY + NUM_STAGES, B_V_EMPTY = B_V_FULL + NUM_STAGES,
   B_S_FULL = B_V_EMPTY + NUM_STAGES,   // [2]
   B_P_FULL = B_S_FULL + 2,             // [2]
@@ -205,6 +210,9 @@ __device__ __forceinline__ int unit_of_round(int r, int cta, int grid, int num_u
 __device__ __forceinline__ int num_rounds(int grid, int num_units) {
   return (num_units + grid - 1) / grid;
 }
+
+// Q slot of tile t in the CTA's ul-th unit.
+__device__ __forceinline__ int q_slot(int ul, int t) { return (2 * ul + t) % Q_SLOTS; }
 
 __device__ __forceinline__ int block_at(const Unit& U, int idx) {
   return idx < U.sb ? idx : U.wlo + (idx - U.sb);
@@ -328,28 +336,38 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
   // Failure-detection test: no copy is issued, so the other roles' bounded
   // waits expire and the CTA reports ATTN_ERR_DEVICE_TIMEOUT and exits.
   if (p.withhold_loads) return;
-  uint32_t q_it = 0, kv_it = 0;
+  uint32_t kv_it = 0;
+  uint32_t q_loads[Q_SLOTS] = {0, 0, 0};
   // parity of the last load issued into each barrier, for the drain
-  int q_last = -1, k_last[NUM_STAGES], v_last[NUM_STAGES];
+  int q_last[Q_SLOTS], k_last[NUM_STAGES], v_last[NUM_STAGES];
+  for (int s = 0; s < Q_SLOTS; ++s) q_last[s] = -1;
   for (int s = 0; s < NUM_STAGES; ++s) k_last[s] = v_last[s] = -1;
   bool ok = true;
+  // one Q tile into its slot, once the MMAs that read the slot before are done
+  auto load_q = [&](const Unit& U, int ul, int t) {
+    const int qs = q_slot(ul, t);
+    const uint32_t ph = q_loads[qs] & 1u;
+    if (!warp_wait(bars + 8 * (B_Q_EMPTY + qs), ph ^ 1u, abort_flag, p)) return false;
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bars + 8 * (B_Q_FULL + qs), G::TILE_BYTES);
+      for (int c = 0; c < G::NCH; ++c)
+        tma_load_3d(sbase + G::Q_OFF + qs * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
+                    bars + 8 * (B_Q_FULL + qs), c * G::CW, U.q0 + t * BM, U.bh);
+    }
+    __syncwarp();
+    q_last[qs] = static_cast<int>(ph);
+    ++q_loads[qs];
+    return true;
+  };
   const int rounds = num_rounds(gridDim.x, p.num_units);
+  int ul = 0;
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     const Unit U = decode_unit(u, p);
-    ok = warp_wait(bars + 8 * B_Q_EMPTY, (q_it & 1u) ^ 1u, abort_flag, p);
+    // Q tile 0 first: its slot was released by the unit before last.
+    ok = load_q(U, ul, 0);
     if (!ok) break;
-    if (elect_one()) {
-      mbar_arrive_expect_tx(bars + 8 * B_Q_FULL, U.n_active * G::TILE_BYTES);
-      for (int t = 0; t < U.n_active; ++t)
-        for (int c = 0; c < G::NCH; ++c)
-          tma_load_3d(sbase + G::Q_OFF + t * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
-                      bars + 8 * B_Q_FULL, c * G::CW, U.q0 + t * BM, U.bh);
-    }
-    __syncwarp();
-    q_last = q_it & 1;
-    ++q_it;
     const int kvz = U.b * p.H_kv + U.g;
     for (int idx = 0; idx < U.n_iter; ++idx, ++kv_it) {
       const int j = block_at(U, idx);
@@ -365,6 +383,12 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       }
       __syncwarp();
       k_last[s] = ph;
+      // Q tile 1 after the first K tile: its slot is the previous unit's
+      // tile-0 slot, free once that unit's last S MMAs are done.
+      if (idx == 0 && U.n_active > 1) {
+        ok = load_q(U, ul, 1);
+        if (!ok) break;
+      }
       ok = warp_wait(bars + 8 * (B_V_EMPTY + s), ph ^ 1u, abort_flag, p);
       if (!ok) break;
       if (elect_one()) {
@@ -376,11 +400,13 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       __syncwarp();
       v_last[s] = ph;
     }
+    ++ul;
   }
   if (!ok) {
-    // Let every copy this thread started land before the CTA can exit.
+    // Let every copy this warp started land before the CTA can exit.
     const unsigned long long lim = p.watchdog_ns;
-    if (q_last >= 0) drain_wait(bars + 8 * B_Q_FULL, q_last, lim);
+    for (int s = 0; s < Q_SLOTS; ++s)
+      if (q_last[s] >= 0) drain_wait(bars + 8 * (B_Q_FULL + s), q_last[s], lim);
     for (int s = 0; s < NUM_STAGES; ++s) {
       if (k_last[s] >= 0) drain_wait(bars + 8 * (B_K_FULL + s), k_last[s], lim);
       if (v_last[s] >= 0) drain_wait(bars + 8 * (B_V_FULL + s), v_last[s], lim);
@@ -389,10 +415,10 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
 }
 
 template <int D, bool BF16>
-__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int t, int stage) {
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t sbase, int t, int qs, int stage) {
   using G = Geo<D>;
   constexpr uint32_t idesc = instr_desc(BF16, BM, BN, false);
-  const uint32_t qa = sbase + G::Q_OFF + t * G::TILE_BYTES;
+  const uint32_t qa = sbase + G::Q_OFF + qs * G::TILE_BYTES;
   const uint32_t ka = sbase + G::K_OFF + stage * G::TILE_BYTES;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
@@ -427,17 +453,39 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int t, i
 template <int D, bool BF16>
 __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
-  uint32_t q_ph = 0, kv_it = 0, p_ph[2] = {0, 0};
+  uint32_t kv_it = 0, p_ph[2] = {0, 0};
+  uint32_t q_uses[Q_SLOTS] = {0, 0, 0};
   bool ok = true;
   const int rounds = num_rounds(gridDim.x, p.num_units);
+  int ul = 0;
+  // S_0 of a unit's first block may already have been issued at the end of
+  // the unit before (see below); its Q tile 0 has then been waited for too.
+  bool s0_pre = false;
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     const Unit U = decode_unit(u, p);
-    ok = warp_wait(bars + 8 * B_Q_FULL, q_ph, abort_flag, p);
-    if (!ok) break;
-    q_ph ^= 1u;
-    tc_fence_after_sync();
+    const int qs0 = q_slot(ul, 0), qs1 = q_slot(ul, 1);
+    auto wait_q = [&](int qs) {
+      if (!warp_wait(bars + 8 * (B_Q_FULL + qs), q_uses[qs] & 1u, abort_flag, p)) return false;
+      ++q_uses[qs];
+      tc_fence_after_sync();
+      return true;
+    };
+    // Q tile t is waited for before its first S MMA of the unit
+    bool q_ready[2] = {s0_pre, false};
+    const bool this_s0_pre = s0_pre;
+    s0_pre = false;
+    auto need_q = [&](int t) {
+      if (q_ready[t]) return true;
+      if (!wait_q(t == 0 ? qs0 : qs1)) return false;
+      q_ready[t] = true;
+      return true;
+    };
+    // the CTA's next unit, for issuing its first S_0 early
+    int u_next = -1;
+    for (int r2 = r + 1; r2 < rounds && u_next < 0; ++r2)
+      u_next = unit_of_round(r2, blockIdx.x, gridDim.x, p.num_units);
     // prologue: S_t for the first block
     {
       const int j0 = block_at(U, 0);
@@ -445,14 +493,24 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       ok = warp_wait(bars + 8 * (B_K_FULL + s), (kv_it / NUM_STAGES) & 1u, abort_flag, p);
       if (!ok) break;
       tc_fence_after_sync();
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (!tile_uses(U, t, j0)) continue;
+        if (t == 0 && this_s0_pre) continue;        // issued at the end of the unit before
+        ok = need_q(t);
+        if (!ok) break;
+        if (elect_one()) {
+          issue_qk<D, BF16>(tmem, sbase, t, t == 0 ? qs0 : qs1, s);
+          mma_commit(bars + 8 * (B_S_FULL + t));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
       if (elect_one()) {
-        for (int t = 0; t < 2; ++t)
-          if (tile_uses(U, t, j0)) {
-            issue_qk<D, BF16>(tmem, sbase, t, s);
-            mma_commit(bars + 8 * (B_S_FULL + t));
-          }
         mma_commit(bars + 8 * (B_K_EMPTY + s));
-        if (U.n_iter == 1) mma_commit(bars + 8 * B_Q_EMPTY);
+        if (U.n_iter == 1) {
+          mma_commit(bars + 8 * (B_Q_EMPTY + qs0));
+          if (U.n_active > 1) mma_commit(bars + 8 * (B_Q_EMPTY + qs1));
+        }
       }
       __syncwarp();
     }
@@ -485,8 +543,10 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         if (!ok) break;
         tc_fence_after_sync();
         if (tile_uses(U, 0, jn)) {
+          ok = need_q(0);
+          if (!ok) break;
           if (elect_one()) {
-            issue_qk<D, BF16>(tmem, sbase, 0, sn);
+            issue_qk<D, BF16>(tmem, sbase, 0, qs0, sn);
             mma_commit(bars + 8 * (B_S_FULL + 0));
           }
           __syncwarp();
@@ -505,20 +565,53 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         __syncwarp();
         ++pv_done[1];
       }
+      if (has_next && tile_uses(U, 1, jn)) {
+        ok = need_q(1);
+        if (!ok) break;
+      }
       if (elect_one()) {
         mma_commit(bars + 8 * (B_V_EMPTY + s));
         if (has_next) {
           if (tile_uses(U, 1, jn)) {
-            issue_qk<D, BF16>(tmem, sbase, 1, sn);
+            issue_qk<D, BF16>(tmem, sbase, 1, qs1, sn);
             mma_commit(bars + 8 * (B_S_FULL + 1));
           }
           mma_commit(bars + 8 * (B_K_EMPTY + sn));
-          if (idx + 2 == U.n_iter) mma_commit(bars + 8 * B_Q_EMPTY);
+          if (idx + 2 == U.n_iter) {
+            // last S MMAs of the unit: both Q slots are free once they are done
+            mma_commit(bars + 8 * (B_Q_EMPTY + qs0));
+            if (U.n_active > 1) mma_commit(bars + 8 * (B_Q_EMPTY + qs1));
+          }
         }
       }
       __syncwarp();
+      // Once Q tile 0 has no block left in this unit (its last P_0 V is
+      // issued and no S_0 follows), its next S is the next unit's first one:
+      // issue it now, so that softmax 0 finds it ready after its epilogue
+      // instead of waiting for tile 1 to finish this unit.  S_0 overwrites
+      // P_0 only after the P_0 V issued before it (the pipe runs in order).
+      if (!s0_pre && u_next >= 0 && has_next && j >= tile_last_block(U, 0) &&
+          idx + 2 == U.n_iter) {
+        const Unit UN = decode_unit(u_next, p);
+        const int jn0 = block_at(UN, 0);
+        if (tile_uses(UN, 0, jn0)) {
+          const uint32_t it2 = kv_it + U.n_iter;       // ring position of the next unit's first K
+          const int s2 = it2 % NUM_STAGES;
+          ok = warp_wait(bars + 8 * (B_K_FULL + s2), (it2 / NUM_STAGES) & 1u, abort_flag, p);
+          if (!ok) break;
+          ok = wait_q(q_slot(ul + 1, 0));
+          if (!ok) break;
+          if (elect_one()) {
+            issue_qk<D, BF16>(tmem, sbase, 0, q_slot(ul + 1, 0), s2);
+            mma_commit(bars + 8 * (B_S_FULL + 0));
+          }
+          __syncwarp();
+          s0_pre = true;
+        }
+      }
     }
     kv_it += U.n_iter;
+    ++ul;
   }
   // Every MMA this warp issued has completed once the drain barrier flips.
   if (elect_one()) mma_commit(bars + 8 * B_DRAIN);
@@ -748,8 +841,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + 8 * B_Q_FULL, 1);
-    mbar_init(bars + 8 * B_Q_EMPTY, 1);
+    for (int s = 0; s < Q_SLOTS; ++s) {
+      mbar_init(bars + 8 * (B_Q_FULL + s), 1);
+      mbar_init(bars + 8 * (B_Q_EMPTY + s), 1);
+    }
     for (int s = 0; s < NUM_STAGES; ++s) {
       mbar_init(bars + 8 * (B_K_FULL + s), 1);
       mbar_init(bars + 8 * (B_K_EMPTY + s), 1);
