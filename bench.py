@@ -11,6 +11,9 @@ workload with inputs resident in HBM.  Prints ONE JSON line on rank 0.
 new row against an 8192-position cache, d=128 bf16) and reports GB/s of
 algorithmic bytes against the measured HBM bandwidth (an extra line).
 
+``--backward`` times attn_bwd (dQ, dK, dV of the same workload's forward) and
+reports TFLOP/s at 10 d flops per kept pair (an extra line).
+
 ``--alibi`` times the same workload through attn_fwd_alibi with the pages'
 slopes 2^(-8 h / H) (an extra measurement, not the headline line; it has no
 host-buffer leg and no CPU-oracle leg).
@@ -390,6 +393,146 @@ def decode_bench(args):
     return 0
 
 
+def backward_bench(args):
+    """--backward: one attn_bwd call (D, the tiled backward, dQ conversion) per
+    timed step on the c3 workload, inputs resident in HBM and rotating over two
+    sets larger than L2.  FLOPs are algorithmic: the five products of the
+    backward (S recomputed, dP, dV, dK, dQ) at 2 d flops per kept pair each,
+    10 d per pair, 2.5 times the forward's count."""
+    import numpy as np
+    import torch
+    import exact_tiled_attention_44_b200 as A
+    import oracle
+    from exact_tiled_attention_44_b200.inputs import WORKLOADS, make_grad_output, make_inputs, to_f64
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    q, k, v = make_inputs(w)
+    do = make_grad_output(w.B, w.H, w.N, w.d, dtype=q.dtype, seed=0)
+    sets = []
+    for i in range(2):
+        qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+        od, ld = A.attention(qd, kd, vd, causal=w.causal, window=w.window, n_sink=w.n_sink,
+                             scale=w.scale)
+        grads = (torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd))
+        ws = torch.empty(A.bwd_workspace_bytes(w.B, w.H, w.N, w.d, A._dtype_code(q)),
+                         dtype=torch.uint8, device=dev)
+        sets.append((qd, kd, vd, od, dod, ld, grads, ws))
+    set_bytes = sum(t.numel() * t.element_size() for t in sets[0][:6])
+    pairs = A.unmasked_pairs(w.N, w.causal, w.window, w.n_sink)
+    flops = 10.0 * w.B * w.H * w.d * pairs
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        qd, kd, vd, od, dod, ld, grads, ws = sets[i % 2]
+        A.attention_backward(qd, kd, vd, od, dod, ld, causal=w.causal, window=w.window,
+                             n_sink=w.n_sink, scale=w.scale, workspace=ws, grads=grads)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0, args.clocks_csv)
+    sampler.start()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    n0 = A.launch_count()
+    sampler.mark_begin()
+    t0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    launches = A.launch_count() - n0
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # end to end through the Python API from pinned host buffers: inputs in,
+    # gradients out, every step
+    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+    ho = sets[0][3].cpu().pin_memory()
+    hl = sets[0][5].cpu().pin_memory()
+    hgrads = tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sets[0][6])
+    qd, kd, vd, od, dod, ld, grads, ws = sets[0]
+
+    def e2e_step():
+        for dst, src in ((qd, hq), (kd, hk), (vd, hv), (od, ho), (dod, hdo), (ld, hl)):
+            dst.copy_(src, non_blocking=True)
+        A.attention_backward(qd, kd, vd, od, dod, ld, causal=w.causal, window=w.window,
+                             n_sink=w.n_sink, scale=w.scale, workspace=ws, grads=grads)
+        for dst, src in zip(hgrads, grads):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(3, min(K, 20))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ho, hdo, hl))
+    d2h = sum(t.numel() * t.element_size() for t in hgrads)
+
+    # the oracle, as it stands, on a bounded sample: whole heads' gradients
+    cpu = None
+    if not args.no_cpu_baseline:
+        t_s, n_heads = 0.0, 0
+        while t_s < 10.0 and n_heads < w.B * w.H:
+            b, h = divmod(n_heads, w.H)
+            g = h // (w.H // w.H_kv)
+            args_h = (to_f64(q[b, h]), to_f64(k[b, g]), to_f64(v[b, g]), to_f64(do[b, h]))
+            c0 = time.perf_counter()
+            oracle.backward_head(*args_h, w.scale, w.causal, w.window, w.n_sink)
+            t_s += time.perf_counter() - c0
+            n_heads += 1
+        cpu = {"value": 10.0 * w.d * pairs * n_heads / t_s / 1e12, "unit": "TFLOP/s",
+               "cores": _blas_threads(), "kind": "oracle",
+               "sample": f"{n_heads} whole heads of {w.name} through oracle.backward_head "
+                         f"(float64, full N x N matrices), {t_s:.1f} s"}
+
+    peaks = load_peaks()
+    achieved = flops / (step_ms / 1e3) / 1e12
+    line = {
+        "metric": "attn bwd TFLOP/s (dQ, dK, dV; 10 d flops per kept pair) & % of measured BF16 peak",
+        "value": flops * K / (total_ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": f"{w.name} backward: B={w.B} H={w.H} H_kv={w.H_kv} N={w.N} d={w.d} "
+                               f"{w.dtype} causal={int(w.causal)}",
+                   "l2": f"inputs larger than L2: 2 rotating sets of {set_bytes / 2**20:.0f} MiB "
+                         "(L2 126 MiB)",
+                   "flops_per_step": flops, "kept_pairs_per_head": pairs,
+                   "outputs": "dq, dk, dv in the input dtype (fp32 dQ accumulator in the workspace)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)",
+                     "kernel_ms": step_ms,
+                     "kernel_ms_scope": "one attn_bwd call: D prep, tiled backward and dQ "
+                                        "conversion launches together (conservative for the "
+                                        "tiled kernel; its share is in the ncu launch list)"},
+        "e2e": {"value": flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": "pinned host q,k,v,o,dO,lse -> device, attention_backward, dq,dk,dv -> host"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "device_status": A.get_status(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -404,6 +547,8 @@ def main():
                     help="time attn_decode on the dec1 workload (GB/s against HBM)")
     ap.add_argument("--alibi", action="store_true",
                     help="add the ALiBi bias with the pages' slopes (attn_fwd_alibi)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time attn_bwd (dQ, dK, dV) on the workload (an extra line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -411,6 +556,8 @@ def main():
         return reference_arm(args)
     if args.decode:
         return decode_bench(args)
+    if args.backward:
+        return backward_bench(args)
 
     import torch
     import exact_tiled_attention_44_b200 as A

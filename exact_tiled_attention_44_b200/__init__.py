@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "AttnError", "attention", "attention_from_host", "attn_fwd_raw", "attn_fwd_alibi_raw",
     "alibi_slopes", "decode", "decode_workspace_bytes", "attn_decode_raw",
-    "attn_decode_noalloc_raw", "unmasked_pairs",
+    "attn_decode_noalloc_raw", "attention_backward", "attn_bwd_raw", "bwd_workspace_bytes",
+    "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
     "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
@@ -41,7 +42,7 @@ EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_s
                     "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
-                    "attn_test_withhold_loads")
+                    "attn_test_withhold_loads", "attn_bwd", "attn_bwd_workspace_bytes")
 
 _LIB = None
 
@@ -94,6 +95,10 @@ def load_library():
     lib.attn_launch_count.restype = ctypes.c_ulonglong
     lib.attn_test_withhold_loads.argtypes = [ci]
     lib.attn_test_withhold_loads.restype = ci
+    lib.attn_bwd.argtypes = [vp] * 11 + [ctypes.c_longlong] + [ci] * 8 + [cf, ci, vp]
+    lib.attn_bwd.restype = ci
+    lib.attn_bwd_workspace_bytes.argtypes = [ci] * 5
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_longlong
     _LIB = lib
     return lib
 
@@ -233,6 +238,72 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = 
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_decode")
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int, dtype: int) -> int:
+    """Scratch bytes attn_bwd needs (dtype: the status-style code incl. ATTN_OUT_F32)."""
+    return int(load_library().attn_bwd_workspace_bytes(B, H, N, d, dtype))
+
+
+def attn_bwd_raw(q, k, v, o, dout, lse, slopes, dq, dk, dv, ws, ws_bytes, B, H, H_kv, N, d,
+                 causal, window, n_sink, scale, dtype, stream) -> int:
+    """Direct C-ABI call of attn_bwd with integer pointers; returns the status code."""
+    return int(load_library().attn_bwd(q, k, v, o, dout, lse, slopes, dq, dk, dv, ws,
+                                       ctypes.c_longlong(ws_bytes), B, H, H_kv, N, d, int(causal),
+                                       window, n_sink, ctypes.c_float(scale), dtype, stream))
+
+
+def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                       dout: torch.Tensor, lse: torch.Tensor, *, causal: bool = False,
+                       window: int = 0, n_sink: int = 0, scale: float | None = None,
+                       alibi_slopes: torch.Tensor | None = None, out_f32: bool = False,
+                       workspace: torch.Tensor | None = None, grads=None):
+    """dQ, dK, dV of attention()'s output for the upstream gradient ``dout``
+    (attn_bwd).  ``o`` and ``dout`` are [B, H, N, d] in q's 16-bit dtype and
+    ``lse`` the forward's float32 [B, H, N]; mask, scale and slopes must be
+    those of the forward.  ``workspace``: CUDA uint8 tensor of at least
+    bwd_workspace_bytes(...) bytes (allocated here with torch when omitted);
+    ``grads``: optional preallocated (dq, dk, dv).  Returns (dq, dk, dv),
+    float32 when ``out_f32``."""
+    _check(q, k, v)
+    if not q.is_cuda:
+        raise ValueError("attention_backward() takes CUDA tensors")
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    for name, t in (("o", o), ("dout", dout)):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor like q")
+    if (lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous()
+            or lse.device != q.device):
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor on q's device")
+    if alibi_slopes is not None:
+        if (alibi_slopes.dtype != torch.float32 or alibi_slopes.device != q.device
+                or tuple(alibi_slopes.shape) != (H,) or not alibi_slopes.is_contiguous()):
+            raise ValueError("alibi_slopes must be a contiguous float32 [H] tensor on q's device")
+    if scale is None:
+        scale = default_scale(d)
+    code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
+    odt = torch.float32 if out_f32 else q.dtype
+    if grads is None:
+        dq = torch.empty((B, H, N, d), dtype=odt, device=q.device)
+        dk = torch.empty((B, H_kv, N, d), dtype=odt, device=q.device)
+        dv = torch.empty((B, H_kv, N, d), dtype=odt, device=q.device)
+    else:
+        dq, dk, dv = grads
+    need = bwd_workspace_bytes(B, H, N, d, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        rc = attn_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                          lse.data_ptr(), alibi_slopes.data_ptr() if alibi_slopes is not None else None,
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws_ptr, ws_bytes, B, H,
+                          H_kv, N, d, causal, window, n_sink, scale, code, stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def _check(q, k, v):

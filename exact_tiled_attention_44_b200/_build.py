@@ -12,7 +12,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "attn_api.cu")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("attn_api.cu", "attn_kernel.cuh", "ptx.cuh")] + [
+DEPS = [os.path.join(PKG, "csrc", f) for f in ("attn_api.cu", "attn_kernel.cuh", "ptx.cuh", "bwd_kernel.cuh",
+                                                   "decode_kernel.cuh")] + [
     os.path.join(ROOT, "include", "attn.h")]
 OUT = os.path.join(PKG, "libattn.so")
 

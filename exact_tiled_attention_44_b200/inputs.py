@@ -130,6 +130,15 @@ def make_decode_inputs(B, H, H_kv, N_q, N_kv, d, dtype=torch.bfloat16, seed=0):
     return tuple(torch.from_numpy(a).to(dtype).contiguous() for a in (q, k, v))
 
 
+def make_grad_output(B, H, N, d, dtype=torch.bfloat16, seed=0):
+    """Upstream gradient dO [B, H, N, d] for the backward pass: float32
+    standard normals from numpy.random.default_rng(seed + 1), rounded to
+    ``dtype`` (seed + 1 keeps it independent of the q, k, v draw of ``seed``)."""
+    rng = np.random.default_rng(seed + 1)
+    g = rng.standard_normal((B, H, N, d), dtype=np.float32)
+    return torch.from_numpy(g).to(dtype).contiguous()
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact float64 upcast of a 16-bit tensor (every bf16/fp16 value is a float64 value)."""
     return t.detach().to("cpu", torch.float64).numpy()

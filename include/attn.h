@@ -36,7 +36,8 @@
  *     (a cudaStream_t passed as void*; NULL = the legacy default stream);
  *     faults inside the kernel surface at the caller's next synchronisation,
  *     and watchdog expiries are reported by attn_get_status().
- *   - Results are deterministic: equal inputs give bitwise-equal outputs.
+ *   - Results are deterministic: equal inputs give bitwise-equal outputs,
+ *     except attn_bwd's dQ (see there).
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -186,6 +187,50 @@ long long attn_decode_workspace_bytes(int B, int H, int H_kv, int N_q, int N_kv,
 int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int H, int H_kv, int N_q, int N_kv, int d, int causal,
                         int window, int n_sink, float scale, int dtype, void* stream);
+
+/*
+ * attn_bwd -- gradients dQ, dK, dV of attn_fwd's output O for an upstream
+ * gradient dO ("USAAIO Lesson 91", slide 9: the Flash Attention 2 backward
+ * recomputes the attention tiles from the saved statistics instead of storing
+ * the N x N matrix).  With P_ij = exp(scale q_i.k_j + bias_ij - LSE_i) over
+ * the kept pairs and D_i = dO_i . O_i:
+ *     dV_j = sum_i P_ij dO_i,   dS_ij = scale P_ij (dO_i . v_j - D_i),
+ *     dQ_i = sum_j dS_ij k_j,   dK_j = sum_i dS_ij q_i,
+ * summed over the query heads of a group for dK and dV.  The pages state no
+ * gradient formula; these are the chain rule through the definition of
+ * attn_fwd, with LSE treated as a saved statistic that receives no gradient.
+ *
+ *   q, k, v   device, as for attn_fwd (16-bit)
+ *   o, dout   device, [B, H, N, d], same 16-bit type: the forward's output and
+ *             the upstream gradient
+ *   lse       device, [B, H, N] float32: the forward's LSE for the same
+ *             q, k, v, mask, scale and slopes
+ *   slopes    device, [H] float32 ALiBi slopes as for attn_fwd_alibi, or NULL
+ *             for no position bias
+ *   dq        device, [B, H, N, d]; dk, dv device, [B, H_kv, N, d]: outputs,
+ *             16-bit, or float32 with ATTN_OUT_F32 in dtype
+ *   workspace, workspace_bytes   device scratch of at least
+ *             attn_bwd_workspace_bytes(B, H, N, d, dtype) bytes, 256-byte
+ *             aligned, owned by the caller; overwritten by the call and not to
+ *             be shared by calls in flight at once
+ * Outputs and workspace must not overlap each other or any input (else
+ * ATTN_ERR_INVALID_ARG); inputs may alias each other.  Sizes, mask, scale,
+ * dtype and the other error conventions are those of attn_fwd.  The call
+ * enqueues three kernels on `stream`: D and the zeroing of the fp32 dQ
+ * accumulator, the tiled backward, and (for 16-bit outputs) the conversion
+ * of dQ.  dQ is summed over key tiles with floating-point atomic adds, so its
+ * last bits may differ between calls with equal inputs; dK and dV are each
+ * written by one CTA and are deterministic.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, const float* slopes, void* dq, void* dk, void* dv,
+             void* workspace, long long workspace_bytes, int B, int H, int H_kv, int N, int d,
+             int causal, int window, int n_sink, float scale, int dtype, void* stream);
+
+/* Host only: bytes of workspace attn_bwd needs (one float per query row, plus
+ * an fp32 dQ accumulator unless dtype has ATTN_OUT_F32), 0 for empty sizes,
+ * -1 for invalid sizes or flags.  Independent of the device. */
+long long attn_bwd_workspace_bytes(int B, int H, int N, int d, int dtype);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_error_string(int status);

@@ -234,3 +234,71 @@ def test_decode_workspace_size():
     assert b >= 8 * 1 * (128 + 1) * 4 * 2
     assert A.decode_workspace_bytes(1, 8, 2, 5, 4, 128) == -1
     assert A.decode_workspace_bytes(0, 8, 2, 1, 4096, 128) == 0
+
+
+# ------------------------------------------------------------------ backward entry point
+
+
+# fake, aligned, never dereferenced addresses (B=1, H=4, N=256, d=64 tensors are 128 KB)
+B_Q, B_K, B_V, B_O, B_DO, B_L, B_S, B_DQ, B_DK, B_DV, B_W = (i << 24 for i in range(1, 12))
+
+
+def call_bwd(**kw):
+    a = dict(q=B_Q, k=B_K, v=B_V, o=B_O, dout=B_DO, lse=B_L, slopes=None, dq=B_DQ, dk=B_DK,
+             dv=B_DV, ws=B_W, ws_bytes=1 << 22, B=1, H=4, H_kv=2, N=256, d=64, causal=1,
+             window=0, n_sink=0, scale=0.125, dtype=A.ATTN_BF16)
+    a.update(kw)
+    return A.attn_bwd_raw(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["slopes"],
+                          a["dq"], a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["B"], a["H"],
+                          a["H_kv"], a["N"], a["d"], a["causal"], a["window"], a["n_sink"],
+                          a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(o=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(dout=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(dk=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), A.ATTN_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), A.ATTN_ERR_INVALID_ARG),            # smaller than the dQ accumulator
+    (dict(ws_bytes=-1), A.ATTN_ERR_INVALID_ARG),
+    (dict(ws=B_W + 16), A.ATTN_ERR_MISALIGNED),               # workspace wants 256 bytes
+    (dict(dout=B_DO + 8), A.ATTN_ERR_MISALIGNED),
+    (dict(lse=B_L + 4), A.ATTN_ERR_MISALIGNED),
+    (dict(slopes=B_S + 2), A.ATTN_ERR_MISALIGNED),
+    (dict(d=48), A.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=0, window=8), A.ATTN_ERR_UNSUPPORTED),
+    (dict(H=6, H_kv=4), A.ATTN_ERR_INVALID_ARG),
+    (dict(dq=B_Q + 256), A.ATTN_ERR_INVALID_ARG),             # dQ overlaps q
+    (dict(dk=B_DV), A.ATTN_ERR_INVALID_ARG),                  # dK overlaps dV
+    (dict(dv=B_L), A.ATTN_ERR_INVALID_ARG),                   # dV overlaps lse
+    (dict(ws=B_DQ), A.ATTN_ERR_INVALID_ARG),                  # workspace overlaps dQ
+    (dict(dq=B_S, slopes=B_S), A.ATTN_ERR_INVALID_ARG),       # dQ overlaps the slopes
+    (dict(scale=float("nan")), A.ATTN_ERR_INVALID_ARG),
+])
+def test_bwd_invalid_calls_are_rejected_before_launch(kw, expect):
+    assert call_bwd(**kw) == expect
+
+
+def test_bwd_inputs_may_alias_each_other():
+    """Read-only inputs may share memory (e.g. o passed as dout); validation
+    then goes on to the device query, which fails here without a GPU."""
+    rc = call_bwd(dout=B_O)
+    assert rc not in (A.ATTN_ERR_INVALID_ARG, A.ATTN_ERR_MISALIGNED, A.ATTN_ERR_UNSUPPORTED)
+
+
+def test_bwd_empty_problem_is_a_no_op():
+    assert call_bwd(B=0, ws=None, ws_bytes=0) == A.ATTN_OK
+    assert call_bwd(N=0, ws=None, ws_bytes=0) == A.ATTN_OK
+
+
+def test_bwd_workspace_size():
+    rows = 2 * 8 * 300
+    # D per row (rounded to 256 bytes), then the fp32 dQ accumulator
+    want = -(-rows * 4 // 256) * 256 + rows * 64 * 4
+    assert A.bwd_workspace_bytes(2, 8, 300, 64, A.ATTN_BF16) == want
+    # fp32 gradients: dQ is accumulated in place, only D remains
+    assert A.bwd_workspace_bytes(2, 8, 300, 64, A.ATTN_BF16 | A.ATTN_OUT_F32) == -(-rows * 4 // 256) * 256
+    assert A.bwd_workspace_bytes(0, 8, 300, 64, A.ATTN_BF16) == 0
+    assert A.bwd_workspace_bytes(-1, 8, 300, 64, A.ATTN_BF16) == -1
+    assert A.bwd_workspace_bytes(1, 8, 300, 64, 0x100) == -1
