@@ -628,7 +628,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   bp.scale_log2 = scale * 1.4426950408889634f;
   bp.scale = scale;
   bp.n_tiles = (N + attn::BN - 1) / attn::BN;
-  const long long units = static_cast<long long>(B) * H_kv * bp.n_tiles;
+  const long long units = static_cast<long long>(B) * H_kv * ((bp.n_tiles + 1) / 2);
   if (units > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
   bp.num_units = static_cast<int>(units);
   bp.alibi = slopes;

@@ -63,7 +63,7 @@ struct BwdParams {
   float scale_log2;    // scale * log2(e)
   float scale;
   int n_tiles;         // ceil(N / 128)
-  int num_units;       // B * H_kv * n_tiles
+  int num_units;       // B * H_kv * ceil(n_tiles / 2) pair units
   const float* alibi;  // ALiBi slope per query head, or nullptr
   int smem_alloc;      // dynamic shared memory bytes given at launch
 };
@@ -89,9 +89,11 @@ struct BwGeo {
   static constexpr uint32_t DK_COL = 128;
   static constexpr uint32_t X_COL = 256;
   static constexpr uint32_t Y_COL = 384;
-  // dQ takes the free half of the dV block when it fits, else X (S^T is dead
-  // once the dV product has read P^T from it).
-  static constexpr uint32_t DQ_COL = D <= 64 ? 64 : X_COL;
+  // dQ takes the free half of the dV block when it fits, else Y: dS^T there
+  // is dead once the dK product (issued before dQ) has read it, and X stays
+  // free for the next tile's S^T, which can then be issued right behind dQ
+  // instead of after the dQ read-out; only the next dP^T waits for that.
+  static constexpr uint32_t DQ_COL = D <= 64 ? 64 : Y_COL;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(G::TILE_BYTES % 1024 == 0, "tiles must stay on swizzle-atom boundaries");
 };
@@ -121,27 +123,49 @@ struct BwUnit {
   int b, g, j, i_lo, n_i, n_steps;
 };
 
-// Unit u: key tile j = u / (B H_kv), so that units are handed out in
-// descending cost order under causality (tile 0 is kept by every query tile).
-// Query tiles visited: i_lo .. i_lo + n_i - 1, the tiles holding a kept pair
-// with key tile j.  Causal: i >= j.  Window: a query keeps a key less than
-// `window` positions behind it, so the last query tile is the one holding
+// Work is handed out in pair units: unit u covers key tiles j = pi and
+// j = n_tiles - 1 - pi of K/V head (b, g), with bg = u / ceil(n_tiles / 2)
+// and pi = u % ceil(n_tiles / 2).  Under causality the two tiles together are
+// kept by n_tiles + 1 query tiles whatever pi is, so every unit costs the
+// same; units are numbered head-major, so the CTAs running at one time share
+// a few heads and their Q, dO and dQ rows stay in L2.  One CTA processes the
+// two key tiles of its unit one after the other (the "halves").
+// For key tile j the query tiles visited are i_lo .. i_lo + n_i - 1, the
+// tiles holding a kept pair with it.  Causal: i >= j.  Window: a query keeps
+// a key less than `window` positions behind it, so the last query tile holds
 // query k0 + 127 + window - 1, unless the key tile holds sink keys (those are
-// kept by every later query).
-__device__ __forceinline__ BwUnit bw_unit(int u, const BwdParams& p) {
+// kept by every later query).  Returns false for the absent second half of a
+// unit whose two tiles coincide (odd n_tiles).
+__device__ __forceinline__ bool bw_unit(int u, int half, const BwdParams& p, BwUnit* out) {
+  const int np = (p.n_tiles + 1) / 2;
+  const int bg = u / np;
+  const int pi = u % np;
+  const int j = half ? p.n_tiles - 1 - pi : pi;
+  if (half && j == pi) return false;
   BwUnit U;
-  const int bg = p.B * p.H_kv;
-  U.j = u / bg;
-  const int r = u % bg;
-  U.b = r / p.H_kv;
-  U.g = r % p.H_kv;
+  U.j = j;
+  U.b = bg / p.H_kv;
+  U.g = bg % p.H_kv;
   U.i_lo = p.causal ? U.j : 0;
   int i_hi = p.n_tiles - 1;
   if (p.window > 0 && U.j * BN >= p.n_sink)
     i_hi = min(i_hi, (U.j * BN + BN - 1 + p.window - 1) / BM);
   U.n_i = i_hi - U.i_lo + 1;
   U.n_steps = U.n_i * (p.H / p.H_kv);
-  return U;
+  *out = U;
+  return true;
+}
+
+// The CTA's key-tile tasks: task k is half k % 2 of the unit the CTA takes in
+// round k / 2.  bw_task returns false for a task the CTA does not have.
+__device__ __forceinline__ int bw_num_tasks(const BwdParams& p) {
+  return 2 * num_rounds(gridDim.x, p.num_units);
+}
+
+__device__ __forceinline__ bool bw_task(int k, const BwdParams& p, BwUnit* U) {
+  const int u = unit_of_round(k >> 1, blockIdx.x, gridDim.x, p.num_units);
+  if (u < 0) return false;
+  return bw_unit(u, k & 1, p, U);
 }
 
 __device__ __forceinline__ void bw_step(const BwUnit& U, const BwdParams& p, int n, int* hq, int* i) {
@@ -198,6 +222,21 @@ __device__ __forceinline__ void bw_tmem_ld(uint32_t taddr, uint32_t (&r)[W]) {
   if constexpr (W == 32) tmem_ld_32x32b_x32(taddr, r);
   else if constexpr (W == 16) tmem_ld_32x32b_x16(taddr, r);
   else bw_tmem_ld_x8(taddr, r);
+}
+
+// ------------------------------------------------------------ shared memory
+
+__device__ __forceinline__ float4 bw_lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void bw_sts(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 // ------------------------------------------------------------ MMA issue
@@ -266,11 +305,10 @@ __device__ void bw_tma_role(const BwdParams& p, const CUtensorMap* tmQ, const CU
   int ul = 0;
   int kv_last = -1, qd_last[2] = {-1, -1};
   bool ok = true;
-  const int rounds = num_rounds(gridDim.x, p.num_units);
-  for (int r = 0; r < rounds && ok; ++r) {
-    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
-    if (u < 0) continue;
-    const BwUnit U = bw_unit(u, p);
+  const int tasks = bw_num_tasks(p);
+  for (int tk = 0; tk < tasks && ok; ++tk) {
+    BwUnit U;
+    if (!bw_task(tk, p, &U)) continue;
     const int kvz = U.b * p.H_kv + U.g;
     ok = bw_warp_wait(bars + 8 * W_KV_EMPTY, (ul & 1) ^ 1, abort_flag, p);
     if (!ok) break;
@@ -288,27 +326,27 @@ __device__ void bw_tma_role(const BwdParams& p, const CUtensorMap* tmQ, const CU
     for (int n = 0; n < U.n_steps; ++n, ++st_it) {
       const int s = st_it & 1;
       const uint32_t ph = (st_it >> 1) & 1u;
-      ok = bw_warp_wait(bars + 8 * (W_QD_EMPTY + s), ph ^ 1u, abort_flag, p);
-      if (!ok) break;
       int hq, i;
       bw_step(U, p, n, &hq, &i);
       const int bh = U.b * p.H + hq;
       const int q0 = i * BM;
-      // statistics of the tile's 128 query rows; rows past N get -inf (P = 0)
-      float* st = reinterpret_cast<float*>(smem + W::ST_OFF + s * W::ST_BYTES);
+      // statistics of the tile's 128 query rows, loaded before the wait for
+      // the stage so that their latency overlaps it; rows past N get LSE = +inf
+      // (P = 0)
+      float nl[4], dd[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int e = lane + 32 * k;
-        const int q = q0 + e;
-        float nl = -INFINITY, dd = 0.f;
+        const int q = q0 + lane + 32 * k;
+        nl[k] = INFINITY;
+        dd[k] = 0.f;
         if (q < p.N) {
           const size_t idx = static_cast<size_t>(bh) * p.N + q;
-          nl = -__ldg(p.lse + idx) * 1.4426950408889634f;
-          dd = __ldg(p.dsum + idx);
+          nl[k] = __ldg(p.lse + idx);
+          dd[k] = __ldg(p.dsum + idx);
         }
-        st[e] = nl;
-        st[128 + e] = dd;
       }
+      ok = bw_warp_wait(bars + 8 * (W_QD_EMPTY + s), ph ^ 1u, abort_flag, p);
+      if (!ok) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(bars + 8 * (W_QD_FULL + s), 2 * G::TILE_BYTES);
         for (int c = 0; c < G::NCH; ++c) {
@@ -319,6 +357,12 @@ __device__ void bw_tma_role(const BwdParams& p, const CUtensorMap* tmQ, const CU
         }
       }
       __syncwarp();
+      const uint32_t st = sbase + W::ST_OFF + s * W::ST_BYTES;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        bw_sts(st + 4 * (lane + 32 * k), -nl[k] * 1.4426950408889634f);
+        bw_sts(st + 4 * (128 + lane + 32 * k), dd[k]);
+      }
       // every lane's statistics stores are released by its own arrival
       mbar_arrive(bars + 8 * (W_QD_FULL + s));
       qd_last[s] = static_cast<int>(ph);
@@ -342,11 +386,10 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
   bool any_dq = false;
   bool ok = true;
   int ul = 0;
-  const int rounds = num_rounds(gridDim.x, p.num_units);
-  for (int r = 0; r < rounds && ok; ++r) {
-    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
-    if (u < 0) continue;
-    const BwUnit U = bw_unit(u, p);
+  const int tasks = bw_num_tasks(p);
+  for (int tk = 0; tk < tasks && ok; ++tk) {
+    BwUnit U;
+    if (!bw_task(tk, p, &U)) continue;
     ok = bw_warp_wait(bars + 8 * W_KV_FULL, ul & 1, abort_flag, p);
     if (!ok) break;
     for (int n = 0; n < U.n_steps; ++n, ++st_it) {
@@ -356,16 +399,20 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
       const uint32_t da = sbase + W::DO_OFF + s * G::TILE_BYTES;
       ok = bw_warp_wait(bars + 8 * (W_QD_FULL + s), ph, abort_flag, p);
       if (!ok) break;
-      if (W::DQ_COL == W::X_COL && any_dq) {
-        // S^T overwrites the previous dQ: wait until it has been read out
-        ok = bw_warp_wait(bars + 8 * W_DQ_FREE, dqf_ph, abort_flag, p);
-        if (!ok) break;
-        dqf_ph ^= 1u;
-      }
       tc_fence_after_sync();
       if (elect_one()) {
         bw_issue_rowdot<D, BF16>(tmem + W::X_COL, sbase + W::K_OFF, qa);
         mma_commit(bars + 8 * W_S_FULL);
+      }
+      __syncwarp();
+      if (W::DQ_COL == W::Y_COL && any_dq) {
+        // dP^T overwrites the previous dQ: wait until it has been read out
+        ok = bw_warp_wait(bars + 8 * W_DQ_FREE, dqf_ph, abort_flag, p);
+        if (!ok) break;
+        dqf_ph ^= 1u;
+        tc_fence_after_sync();
+      }
+      if (elect_one()) {
         bw_issue_rowdot<D, BF16>(tmem + W::Y_COL, sbase + W::V_OFF, da);
         mma_commit(bars + 8 * W_DP_FULL);
       }
@@ -385,7 +432,7 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
       ok = bw_warp_wait(bars + 8 * W_DS_FULL, ds_ph, abort_flag, p);
       if (!ok) break;
       ds_ph ^= 1u;
-      if (W::DQ_COL != W::X_COL && any_dq) {
+      if (W::DQ_COL != W::Y_COL && any_dq) {
         ok = bw_warp_wait(bars + 8 * W_DQ_FREE, dqf_ph, abort_flag, p);
         if (!ok) break;
         dqf_ph ^= 1u;
@@ -454,11 +501,10 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
   const uint32_t ds_row = sbase + W::DS_OFF + wg * W::DS_CHUNK + t * 128;
   uint32_t st_it = 0, s_ph = 0, dp_ph = 0, dq_ph = 0, acc_ph = 0;
   bool ok = true;
-  const int rounds = num_rounds(gridDim.x, p.num_units);
-  for (int r = 0; r < rounds && ok; ++r) {
-    const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
-    if (u < 0) continue;
-    const BwUnit U = bw_unit(u, p);
+  const int tasks = bw_num_tasks(p);
+  for (int tk = 0; tk < tasks && ok; ++tk) {
+    BwUnit U;
+    if (!bw_task(tk, p, &U)) continue;
     const int k0 = U.j * BN;
     const int kt = k0 + t;
     for (int n = 0; n < U.n_steps; ++n, ++st_it) {
@@ -469,8 +515,8 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       const int q0 = i * BM;
       const int qc = q0 + 64 * wg;           // first query of this warpgroup's columns
       const bool masked = bw_needs_mask(p, q0, k0);
-      const float* nl = reinterpret_cast<const float*>(smem + W::ST_OFF + s * W::ST_BYTES) + 64 * wg;
-      const float* dd = nl + 128;
+      const uint32_t nl = sbase + W::ST_OFF + s * W::ST_BYTES + 4 * 64 * wg;   // -LSE log2(e)
+      const uint32_t dd = nl + 4 * 128;                                        // D
       ok = bw_wait(bars + 8 * (W_QD_FULL + s), ph, abort_flag, p);
       if (!ok) break;
       ok = bw_wait(bars + 8 * W_S_FULL, s_ph, abort_flag, p);
@@ -483,7 +529,7 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       if (!masked && !ALIBI) {
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(nl + e);
+          const float4 l4 = bw_lds4(nl + 4 * e);
           const float2 a = fma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2,
                                 make_float2(l4.x, l4.y));
           const float2 b = fma2(make_float2(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])),
@@ -496,9 +542,14 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       } else {
         const float slope2 = ALIBI ? p.alibi[hq] * 1.4426950408889634f : 0.f;
         const float rel = static_cast<float>(qc - kt);   // (query - key) at column 0, exact
+        float nle[4];
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
-          float x = fmaf(__uint_as_float(sr[e]), c, nl[e]);
+          if ((e & 3) == 0) {
+            const float4 l4 = bw_lds4(nl + 4 * e);
+            nle[0] = l4.x; nle[1] = l4.y; nle[2] = l4.z; nle[3] = l4.w;
+          }
+          float x = fmaf(__uint_as_float(sr[e]), c, nle[e & 3]);
           if constexpr (ALIBI) x = fmaf(-slope2, fabsf(rel + static_cast<float>(e)), x);
           if (masked && !bw_kept(p, qc + e, kt)) x = -INFINITY;
           pv[e] = fast_exp2(x);
@@ -524,7 +575,7 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(dd + e);
+          const float4 d4 = bw_lds4(dd + 4 * e);
           const float2 ta = sub2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
                                  make_float2(d4.x, d4.y));
           const float2 tb = sub2(make_float2(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])),
@@ -556,19 +607,34 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       dq_ph ^= 1u;
       tc_fence_after_sync();
       {
-        const int q = q0 + t;
-        float* dst = p.dq_acc + (static_cast<size_t>(U.b * p.H + hq) * p.N + q) * D + wg * HD;
+        // Each warp turns its 32 rows x OC columns around through its own
+        // slice of the dS tile (rows 32 w4 .. 32 w4 + 31 of chunk wg, free once
+        // the dQ product has read it), so that the atomic adds of one
+        // instruction cover whole 128-byte lines of a few rows instead of 16
+        // bytes of 32 rows.
+        constexpr int UPR = OC / 4;          // 16-byte units per staged row
+        constexpr int RPI = 32 / UPR;        // rows per read-back instruction
+        const uint32_t stg = ds_row - lane * 128;   // this warp's 4 KB slice
+        const size_t row0 = static_cast<size_t>(U.b * p.H + hq) * p.N + q0 + w4 * 32;
 #pragma unroll
         for (int cc = 0; cc < HD / OC; ++cc) {
           uint32_t v[OC];
           bw_tmem_ld<OC>(dq_t + cc * OC, v);
-          if (q < p.N) {
 #pragma unroll
-            for (int e = 0; e < OC; e += 4)
-              atomicAdd(reinterpret_cast<float4*>(dst + cc * OC + e),
-                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                    __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])));
+          for (int un = 0; un < UPR; ++un)
+            st_shared_v4(stg + lane * (OC * 4) + ((un ^ (lane & (UPR - 1))) << 4), v[4 * un],
+                         v[4 * un + 1], v[4 * un + 2], v[4 * un + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < UPR; ++k) {
+            const int r = k * RPI + lane / UPR;
+            const int un = lane % UPR;
+            const float4 x = bw_lds4(stg + r * (OC * 4) + ((un ^ (r & (UPR - 1))) << 4));
+            if (q0 + w4 * 32 + r < p.N)
+              atomicAdd(reinterpret_cast<float4*>(p.dq_acc + (row0 + r) * D + wg * HD + cc * OC +
+                                                  4 * un), x);
           }
+          __syncwarp();
         }
       }
       tc_fence_before_sync();
