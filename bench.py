@@ -49,9 +49,13 @@ KERNEL_SOURCES = ["exact_tiled_attention_44_b200/csrc/attn_kernel.cuh",
                   "exact_tiled_attention_44_b200/csrc/ptx.cuh"]
 
 
-def kernel_source_hash() -> str:
+# device code of the backward kernel (it builds on the forward's helpers)
+BWD_KERNEL_SOURCES = ["exact_tiled_attention_44_b200/csrc/bwd_kernel.cuh"] + KERNEL_SOURCES
+
+
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (sources or KERNEL_SOURCES):
         h.update(open(os.path.join(ROOT, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -66,13 +70,14 @@ def load_peaks():
             "source": "fallback"}
 
 
-def load_traffic(workload: str):
+def load_traffic(workload: str, kind: str = "fwd"):
     """DRAM bytes per launch from the committed ncu summary, if it matches this kernel."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}_traffic.json")
+    path = os.path.join(ROOT, "profiles", f"attn_{kind}_{workload}_traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path))
-    if d.get("kernel_src_sha256") != kernel_source_hash():
+    srcs = BWD_KERNEL_SOURCES if kind == "bwd" else KERNEL_SOURCES
+    if d.get("kernel_src_sha256") != kernel_source_hash(srcs):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -514,7 +519,8 @@ def backward_bench(args):
                    "outputs": "dq, dk, dv in the input dtype (fp32 dQ accumulator in the workspace)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None,
+                     "traffic": load_traffic(w.name, "bwd"),
+                     "traffic_scope": "DRAM bytes of one launch of the tiled backward kernel",
                      "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)",
                      "kernel_ms": step_ms,
                      "kernel_ms_scope": "one attn_bwd call: D prep, tiled backward and dQ "
