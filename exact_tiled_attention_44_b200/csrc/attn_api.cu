@@ -529,10 +529,25 @@ int validate_bwd(const void* q, const void* k, const void* v, const void* o, con
   return ATTN_OK;
 }
 
+// 3-D view [B*H][N][d] of the fp32 dQ buffer for the backward's bulk
+// reductions: 32 x 32 boxes, 128-byte swizzle (d >= 64 only).
+int encode_dq_map(CUtensorMap* map, void* base, int d, int n, int z) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                              static_cast<cuuint64_t>(z)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(n) * d * 4};
+  const cuuint32_t box[3] = {32u, 32u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 template <int D, bool BF16, bool F32, bool ALIBI>
 int launch_bwd_main(DeviceState* st, const CUtensorMap& mq, const CUtensorMap& mk,
-                    const CUtensorMap& mv, const CUtensorMap& mdo, attn::BwdParams bp,
-                    cudaStream_t stream) {
+                    const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdq,
+                    attn::BwdParams bp, cudaStream_t stream) {
   auto kern = attn::attn_bwd_kernel<D, BF16, F32, ALIBI>;
   const int need = attn::BwGeo<D>::SMEM_BYTES;
   // room for aligning the base to 1024 bytes where it fits; at least half of
@@ -557,7 +572,7 @@ int launch_bwd_main(DeviceState* st, const CUtensorMap& mq, const CUtensorMap& m
   }
   bp.smem_alloc = smem;
   const int grid = bp.num_units < st->sm_count ? bp.num_units : st->sm_count;
-  kern<<<grid, attn::BW_THREADS, smem, stream>>>(mq, mk, mv, mdo, bp);
+  kern<<<grid, attn::BW_THREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, bp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -565,7 +580,8 @@ int launch_bwd_main(DeviceState* st, const CUtensorMap& mq, const CUtensorMap& m
 template <int D, bool BF16>
 int launch_bwd_d(DeviceState* st, bool f32, bool alibi, const void* o, const void* dout,
                  void* dq, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                 const CUtensorMap& mdo, attn::BwdParams bp, long long rows, cudaStream_t s) {
+                 const CUtensorMap& mdo, const CUtensorMap& mdq, attn::BwdParams bp,
+                 long long rows, cudaStream_t s) {
   // 1. D = rowsum(dO * O); zero the fp32 dQ accumulator
   const long long blocks = (rows + 7) / 8;
   if (blocks > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
@@ -575,10 +591,10 @@ int launch_bwd_d(DeviceState* st, bool f32, bool alibi, const void* o, const voi
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   // 2. the tiled backward
   int rc;
-  if (f32) rc = alibi ? launch_bwd_main<D, BF16, true, true>(st, mq, mk, mv, mdo, bp, s)
-                      : launch_bwd_main<D, BF16, true, false>(st, mq, mk, mv, mdo, bp, s);
-  else rc = alibi ? launch_bwd_main<D, BF16, false, true>(st, mq, mk, mv, mdo, bp, s)
-                  : launch_bwd_main<D, BF16, false, false>(st, mq, mk, mv, mdo, bp, s);
+  if (f32) rc = alibi ? launch_bwd_main<D, BF16, true, true>(st, mq, mk, mv, mdo, mdq, bp, s)
+                      : launch_bwd_main<D, BF16, true, false>(st, mq, mk, mv, mdo, mdq, bp, s);
+  else rc = alibi ? launch_bwd_main<D, BF16, false, true>(st, mq, mk, mv, mdo, mdq, bp, s)
+                  : launch_bwd_main<D, BF16, false, false>(st, mq, mk, mv, mdo, mdq, bp, s);
   if (rc != ATTN_OK || f32) return rc;
   // 3. dQ to the 16-bit output
   const long long n4 = rows * D / 4;
@@ -614,6 +630,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   bp.lse = lse;
   bp.dsum = reinterpret_cast<float*>(w);
   bp.dq_acc = f32 ? static_cast<float*>(dq) : reinterpret_cast<float*>(w + pl.dq_off);
+  alignas(64) CUtensorMap mdq;
+  std::memset(&mdq, 0, sizeof(mdq));   // unused below d = 64 (atomics path)
+  if (d >= 64 && encode_dq_map(&mdq, bp.dq_acc, d, N, B * H) != ATTN_OK) return ATTN_ERR_CUDA;
   bp.dk = dk;
   bp.dv = dv;
   bp.status = st->status;
@@ -636,14 +655,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool al = slopes != nullptr;
   switch (d) {
-    case 16: return bf16 ? launch_bwd_d<16, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s)
-                         : launch_bwd_d<16, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s);
-    case 32: return bf16 ? launch_bwd_d<32, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s)
-                         : launch_bwd_d<32, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s);
-    case 64: return bf16 ? launch_bwd_d<64, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s)
-                         : launch_bwd_d<64, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s);
-    case 128: return bf16 ? launch_bwd_d<128, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s)
-                          : launch_bwd_d<128, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, bp, rows, s);
+    case 16: return bf16 ? launch_bwd_d<16, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s)
+                         : launch_bwd_d<16, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s);
+    case 32: return bf16 ? launch_bwd_d<32, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s)
+                         : launch_bwd_d<32, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s);
+    case 64: return bf16 ? launch_bwd_d<64, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s)
+                         : launch_bwd_d<64, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s);
+    case 128: return bf16 ? launch_bwd_d<128, true>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s)
+                          : launch_bwd_d<128, false>(st, f32, al, o, dout, dq, mq, mk, mv, mdo, mdq, bp, rows, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }

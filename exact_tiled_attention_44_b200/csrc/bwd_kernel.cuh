@@ -80,7 +80,7 @@ struct BwGeo {
   // 128-byte swizzle (the MN-major operand layout).
   static constexpr int DS_CHUNK = 128 * 128;
   static constexpr int DS_BYTES = 2 * DS_CHUNK;
-  // per stage: 128 floats -LSE*log2(e), then 128 floats D
+  // per stage: 128 floats -LSE*log2(e), then 128 floats -scale*D
   static constexpr int ST_OFF = DS_OFF + DS_BYTES;
   static constexpr int ST_BYTES = 2 * 128 * 4;
   static constexpr int BAR_OFF = ST_OFF + 2 * ST_BYTES;
@@ -239,6 +239,33 @@ __device__ __forceinline__ void bw_sts(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+// ------------------------------------------------------------ bulk reduction
+
+// Adds a box of fp32 values from shared memory into global memory (the TMA
+// unit performs the read-modify-write in L2); completion is tracked per
+// issuing thread by bulk groups.
+__device__ __forceinline__ void bw_tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int x,
+                                                     int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void bw_bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until this thread's bulk operations have finished reading shared memory.
+__device__ __forceinline__ void bw_bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until this thread's bulk operations have completed.
+__device__ __forceinline__ void bw_bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------ MMA issue
 
 // kind::f16 instruction descriptor with both operand major-ness bits (bit 15:
@@ -361,7 +388,7 @@ __device__ void bw_tma_role(const BwdParams& p, const CUtensorMap* tmQ, const CU
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         bw_sts(st + 4 * (lane + 32 * k), -nl[k] * 1.4426950408889634f);
-        bw_sts(st + 4 * (128 + lane + 32 * k), dd[k]);
+        bw_sts(st + 4 * (128 + lane + 32 * k), -p.scale * dd[k]);
       }
       // every lane's statistics stores are released by its own arrival
       mbar_arrive(bars + 8 * (W_QD_FULL + s));
@@ -483,8 +510,8 @@ __device__ __forceinline__ void bw_store_row(void* base, size_t off, const uint3
 }
 
 template <int D, bool BF16, bool OUT_F32, bool ALIBI>
-__device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem, uint32_t sbase,
-                                uint32_t bars, int wg, int w4, int lane,
+__device__ void bw_compute_role(const BwdParams& p, const CUtensorMap* tmDQ, uint32_t tmem,
+                                uint32_t sbase, uint32_t bars, int wg, int w4, int lane,
                                 volatile int* abort_flag) {
   using W = BwGeo<D>;
   constexpr int HD = D / 2;               // output columns of this warpgroup
@@ -500,6 +527,7 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
   // dS tile row t (key), chunk wg (this warpgroup's 64 queries)
   const uint32_t ds_row = sbase + W::DS_OFF + wg * W::DS_CHUNK + t * 128;
   uint32_t st_it = 0, s_ph = 0, dp_ph = 0, dq_ph = 0, acc_ph = 0;
+  bool stg_busy = false;   // a dQ bulk reduction may still read this warp's dS slice
   bool ok = true;
   const int tasks = bw_num_tasks(p);
   for (int tk = 0; tk < tasks && ok; ++tk) {
@@ -516,7 +544,7 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       const int qc = q0 + 64 * wg;           // first query of this warpgroup's columns
       const bool masked = bw_needs_mask(p, q0, k0);
       const uint32_t nl = sbase + W::ST_OFF + s * W::ST_BYTES + 4 * 64 * wg;   // -LSE log2(e)
-      const uint32_t dd = nl + 4 * 128;                                        // D
+      const uint32_t dd = nl + 4 * 128;                                        // -scale D
       ok = bw_wait(bars + 8 * (W_QD_FULL + s), ph, abort_flag, p);
       if (!ok) break;
       ok = bw_wait(bars + 8 * W_S_FULL, s_ph, abort_flag, p);
@@ -576,16 +604,24 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
           const float4 d4 = bw_lds4(dd + 4 * e);
-          const float2 ta = sub2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
-                                 make_float2(d4.x, d4.y));
-          const float2 tb = sub2(make_float2(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])),
-                                 make_float2(d4.z, d4.w));
-          const float2 ga = mul2(mul2(make_float2(pv[e], pv[e + 1]), sc2), ta);
-          const float2 gb = mul2(mul2(make_float2(pv[e + 2], pv[e + 3]), sc2), tb);
+          // dS = P (scale dP - scale D)
+          const float2 ta = fma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
+                                 sc2, make_float2(d4.x, d4.y));
+          const float2 tb = fma2(make_float2(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])),
+                                 sc2, make_float2(d4.z, d4.w));
+          const float2 ga = mul2(make_float2(pv[e], pv[e + 1]), ta);
+          const float2 gb = mul2(make_float2(pv[e + 2], pv[e + 3]), tb);
           pk[e / 2] = pack2<BF16>(ga.x, ga.y);
           pk[e / 2 + 1] = pack2<BF16>(gb.x, gb.y);
         }
         tmem_st_32x32b_x32(y_t, pk);
+        // the warp's slice of the dS tile may still be read by its last dQ
+        // bulk reduction
+        if (stg_busy) {
+          if (lane == 0) bw_bulk_wait_read();
+          __syncwarp();
+          stg_busy = false;
+        }
         // the same 64 values into the dS tile: 8 16-byte units, 128-byte swizzle
 #pragma unroll
         for (int un = 0; un < 8; ++un)
@@ -606,15 +642,45 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
       if (!ok) break;
       dq_ph ^= 1u;
       tc_fence_after_sync();
-      {
-        // Each warp turns its 32 rows x OC columns around through its own
-        // slice of the dS tile (rows 32 w4 .. 32 w4 + 31 of chunk wg, free once
-        // the dQ product has read it), so that the atomic adds of one
-        // instruction cover whole 128-byte lines of a few rows instead of 16
-        // bytes of 32 rows.
+      if constexpr (OC == 32) {
+        // Each warp stages its 32 rows x 32 columns of dQ in its own 4 KB slice
+        // of the dS tile (rows 32 w4 .. 32 w4 + 31 of chunk wg, free once the
+        // dQ product has read it) in the 128-byte swizzle of the dQ tensor map,
+        // and one lane adds the box to the fp32 dQ buffer with a TMA bulk
+        // reduction.  The lane waits for the box to be read out of shared
+        // memory only before the slice is written again.
+        const uint32_t stg = ds_row - lane * 128;
+        const int r0 = q0 + w4 * 32;
+#pragma unroll
+        for (int cc = 0; cc < HD / OC; ++cc) {
+          uint32_t v[OC];
+          bw_tmem_ld<OC>(dq_t + cc * OC, v);
+          if (stg_busy) {
+            if (lane == 0) bw_bulk_wait_read();
+            __syncwarp();
+            stg_busy = false;
+          }
+#pragma unroll
+          for (int un = 0; un < 8; ++un)
+            st_shared_v4(stg + lane * 128 + ((un ^ (lane & 7)) << 4), v[4 * un], v[4 * un + 1],
+                         v[4 * un + 2], v[4 * un + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (r0 < p.N) {
+            if (lane == 0) {
+              bw_tma_reduce_add_3d(tmDQ, stg, wg * HD + cc * OC, r0, U.b * p.H + hq);
+              bw_bulk_commit();
+            }
+            stg_busy = true;
+          }
+        }
+      } else {
+        // Narrow heads: each warp turns its 32 rows x OC columns around
+        // through its own slice of the dS tile, so that the atomic adds of one
+        // instruction cover whole rows instead of 16 bytes of 32 rows.
         constexpr int UPR = OC / 4;          // 16-byte units per staged row
         constexpr int RPI = 32 / UPR;        // rows per read-back instruction
-        const uint32_t stg = ds_row - lane * 128;   // this warp's 4 KB slice
+        const uint32_t stg = ds_row - lane * 128;   // this warp's slice
         const size_t row0 = static_cast<size_t>(U.b * p.H + hq) * p.N + q0 + w4 * 32;
 #pragma unroll
         for (int cc = 0; cc < HD / OC; ++cc) {
@@ -662,13 +728,16 @@ __device__ void bw_compute_role(const BwdParams& p, uint32_t tmem, uint8_t* smem
     __syncwarp();
     if (lane == 0) mbar_arrive(bars + 8 * W_ACC_FREE);
   }
+  // the dQ reductions this warp issued complete before the CTA exits
+  if (lane == 0) bw_bulk_wait_all();
+  __syncwarp();
 }
 
 template <int D, bool BF16, bool OUT_F32, bool ALIBI>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using W = BwGeo<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
@@ -725,8 +794,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // warps under different register budgets would have to fit the smaller).
   if (warp < BW_COMPUTE_WARPS) {
     regs_increase<BW_COMPUTE_REGS>();
-    bw_compute_role<D, BF16, OUT_F32, ALIBI>(p, tmem, smem, sbase, bars, warp / 4, warp % 4, lane,
-                                            abort_flag);
+    bw_compute_role<D, BF16, OUT_F32, ALIBI>(p, &tmDQ, tmem, sbase, bars, warp / 4, warp % 4,
+                                            lane, abort_flag);
     tc_fence_before_sync();
     __syncthreads();
   } else {
