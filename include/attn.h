@@ -1,5 +1,7 @@
 /*
- * attn.h -- C ABI of the exact tiled attention forward library (libattn.so).
+ * attn.h -- C ABI of the exact tiled attention library (libattn.so): the
+ * forward (attn_fwd, attn_fwd_alibi, attn_fwd_host), its backward (attn_bwd) and
+ * the split-KV decoding step (attn_decode, attn_decode_noalloc).
  *
  * The library computes, for every batch b and query head h,
  *
