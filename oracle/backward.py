@@ -89,3 +89,43 @@ def attention_backward(Q, K, V, dO, scale, causal=False, window=0, n_sink=0, slo
 def row_dot(O, dO):
     """D_i = dO_i . O_i per query row ([B, H, N]): the row term of dS."""
     return (np.asarray(O, np.float64) * np.asarray(dO, np.float64)).sum(axis=-1)
+
+
+def tiled_backward_head(q, k, v, o, do, lse, scale, causal, window=0, n_sink=0, slope=0.0,
+                        bs=16):
+    """dQ, dK, dV of one head by the tiled recomputation the pages name for
+    the Flash Attention 2 backward ("USAAIO Lesson 91", slide 9: the attention
+    tiles are recomputed from saved statistics instead of being stored).
+
+    Key blocks outside, query blocks inside.  The saved statistics are the
+    forward's output ``o`` and natural-log ``lse``; for each block pair the
+    probabilities are recomputed as P = exp(s - LSE) (0 where masked), and
+    D_i = dO_i . o_i.  dK and dV of a key block are complete after its inner
+    loop; dQ is summed over key blocks.  Ragged last blocks are allowed.
+    Float64 throughout.  Used only to pin ``backward_head`` (and to state the
+    recomputation in code); it produces no expected value for the GPU.
+    """
+    q, k, v, o, do = (np.asarray(x, np.float64) for x in (q, k, v, o, do))
+    lse = np.asarray(lse, np.float64)
+    n = k.shape[0]
+    d_row = (do * o).sum(axis=1)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for c0 in range(0, n, bs):
+        cols = np.arange(c0, min(n, c0 + bs))
+        for r0 in range(0, q.shape[0], bs):
+            rows = np.arange(r0, min(q.shape[0], r0 + bs))
+            keep = keep_mask(n, n, causal, window, n_sink, rows)[:, cols]
+            if not keep.any():
+                continue
+            s = float(scale) * (q[rows] @ k[cols].T)
+            if slope:
+                s = s - float(slope) * np.abs(rows[:, None] - cols[None, :])
+            p = np.exp(np.where(keep, s - lse[rows][:, None], -np.inf))
+            dv[cols] += p.T @ do[rows]
+            dp = do[rows] @ v[cols].T
+            ds = p * (dp - d_row[rows][:, None])
+            dq[rows] += float(scale) * (ds @ k[cols])
+            dk[cols] += float(scale) * (ds.T @ q[rows])
+    return dq, dk, dv

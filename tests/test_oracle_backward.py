@@ -230,3 +230,23 @@ def test_row_dot_matches_forward():
         P = oracle.attention_weights(q[0, h], k[0, h], 0.4, True)
         dP = do[0, h] @ v[0, h].T
         assert np.abs((P * dP).sum(1) - D[0, h]).max() < 1e-12
+
+
+@pytest.mark.parametrize("bs", [1, 5, 16, 64])
+def test_tiled_recomputation_equals_the_definition(bs):
+    """The tiled recomputation from the saved (O, LSE) of the forward (slide 9)
+    reaches the plain gradients to rounding, for every mask kind, ALiBi and a
+    block size that does not divide N."""
+    q, k, v, do = _inputs(1, 2, 1, 41, 6, seed=17)
+    sl = oracle.alibi_slopes(2)
+    for causal, w, ns, alibi in CASES:
+        for h in range(2):
+            slope = float(sl[h]) if alibi else 0.0
+            O, L = oracle.attention_head(q[0, h], k[0, 0], v[0, 0], 0.6, causal, w, ns,
+                                         slope=slope)
+            want = oracle.backward_head(q[0, h], k[0, 0], v[0, 0], do[0, h], 0.6, causal, w, ns,
+                                        slope)
+            got = oracle.tiled_backward_head(q[0, h], k[0, 0], v[0, 0], O, do[0, h], L, 0.6,
+                                             causal, w, ns, slope, bs=bs)
+            for a, b in zip(got, want):
+                assert np.abs(a - b).max() < 1e-12 * max(1.0, np.abs(b).max())
