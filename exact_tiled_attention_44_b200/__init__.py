@@ -211,13 +211,21 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = 
         raise ValueError(f"shape mismatch q={tuple(q.shape)} k={tuple(k.shape)}")
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share one dtype")
-    if not q.is_cuda:
-        raise ValueError("decode() takes CUDA tensors")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
     for t in (q, k, v):
         if not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous")
     B, H, N_q, d = q.shape
     H_kv, N_kv = k.shape[1], k.shape[2]
+    if out is not None:
+        _expect(out, "out", (B, H, N_q, d), torch.float32 if out_f32 else q.dtype, q.device)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N_q), torch.float32, q.device)
+    if workspace is not None:
+        _expect_workspace(workspace, q.device)
+    if not q.is_cuda:
+        raise ValueError("decode() takes CUDA tensors")
     if scale is None:
         scale = default_scale(d)
     code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
@@ -266,8 +274,6 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     ``grads``: optional preallocated (dq, dk, dv).  Returns (dq, dk, dv),
     float32 when ``out_f32``."""
     _check(q, k, v)
-    if not q.is_cuda:
-        raise ValueError("attention_backward() takes CUDA tensors")
     B, H, N, d = q.shape
     H_kv = k.shape[1]
     for name, t in (("o", o), ("dout", dout)):
@@ -280,10 +286,20 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
         if (alibi_slopes.dtype != torch.float32 or alibi_slopes.device != q.device
                 or tuple(alibi_slopes.shape) != (H,) or not alibi_slopes.is_contiguous()):
             raise ValueError("alibi_slopes must be a contiguous float32 [H] tensor on q's device")
+    odt = torch.float32 if out_f32 else q.dtype
+    if grads is not None:
+        if len(grads) != 3:
+            raise ValueError("grads must be (dq, dk, dv)")
+        _expect(grads[0], "dq", (B, H, N, d), odt, q.device)
+        _expect(grads[1], "dk", (B, H_kv, N, d), odt, q.device)
+        _expect(grads[2], "dv", (B, H_kv, N, d), odt, q.device)
+    if workspace is not None:
+        _expect_workspace(workspace, q.device)
+    if not q.is_cuda:
+        raise ValueError("attention_backward() takes CUDA tensors")
     if scale is None:
         scale = default_scale(d)
     code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
-    odt = torch.float32 if out_f32 else q.dtype
     if grads is None:
         dq = torch.empty((B, H, N, d), dtype=odt, device=q.device)
         dk = torch.empty((B, H_kv, N, d), dtype=odt, device=q.device)
@@ -313,10 +329,28 @@ def _check(q, k, v):
         raise ValueError(f"shape mismatch q={tuple(q.shape)} k={tuple(k.shape)} v={tuple(v.shape)}")
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k, v must share one dtype")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
     _dtype_code(q)
     for t in (q, k, v):
         if not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous")
+
+
+def _expect(t: torch.Tensor, name: str, shape, dtype, device=None):
+    """Caller-provided buffers must match what the C ABI will write: it sizes
+    every tensor from B, H, H_kv, N and d alone."""
+    if (tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous()
+            or (device is not None and t.device != device)):
+        where = f" on {device}" if device is not None else ""
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}{where}, "
+                         f"got {tuple(t.shape)} {t.dtype} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _expect_workspace(ws: torch.Tensor, device):
+    if ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous() or ws.device != device:
+        raise ValueError(f"workspace must be a contiguous 1-D uint8 tensor on {device}")
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
@@ -333,10 +367,14 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool
     [B, H, N] float32 (None when ``return_lse`` is False).
     """
     _check(q, k, v)
-    if not q.is_cuda:
-        raise ValueError("attention() takes CUDA tensors; use attention_from_host() for host tensors")
     B, H, N, d = q.shape
     H_kv = k.shape[1]
+    if out is not None:
+        _expect(out, "out", (B, H, N, d), torch.float32 if out_f32 else q.dtype, q.device)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N), torch.float32, q.device)
+    if not q.is_cuda:
+        raise ValueError("attention() takes CUDA tensors; use attention_from_host() for host tensors")
     if scale is None:
         scale = default_scale(d)
     code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
@@ -378,10 +416,25 @@ def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, st
     _check(q, k, v)
     B, H, N, d = q.shape
     H_kv = k.shape[1]
+    odt = torch.float32 if out_f32 else q.dtype
+    cpu = torch.device("cpu")
+    _expect(out, "out", (B, H, N, d), odt, cpu)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N), torch.float32, cpu)
+        if staging.get("lse") is None:
+            raise ValueError("staging needs an 'lse' tensor when lse is requested")
+    dev = staging["q"].device
+    _expect(staging["q"], "staging['q']", q.shape, q.dtype, dev)
+    _expect(staging["k"], "staging['k']", k.shape, k.dtype, dev)
+    _expect(staging["v"], "staging['v']", v.shape, v.dtype, dev)
+    _expect(staging["o"], "staging['o']", (B, H, N, d), odt, dev)
+    if staging.get("lse") is not None:
+        _expect(staging["lse"], "staging['lse']", (B, H, N), torch.float32, dev)
+    if dev.type != "cuda":
+        raise ValueError("staging tensors must be CUDA tensors")
     if scale is None:
         scale = default_scale(d)
     code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
-    dev = staging["q"].device
     s = (stream or torch.cuda.current_stream(dev)).cuda_stream
     dl = staging.get("lse")
     with torch.cuda.device(dev):
