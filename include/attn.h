@@ -248,7 +248,8 @@ long long attn_unmasked_pairs(int N, int causal, int window, int n_sink);
 
 /*
  * attn_visited_blocks -- host only: the number of (128-query-row block,
- * 128-key block) pairs the kernel's schedule computes for one head.  A block
+ * 128-key block) pairs the kernel's schedule computes for one head (the same
+ * set for the forward and for attn_bwd).  A block
  * pair is visited iff it holds at least one kept pair (causal, window and sink
  * skipping as in Lab 3's "only key blocks at or before this query block").
  * Returns -1 for invalid arguments.
@@ -260,7 +261,11 @@ long long attn_visited_blocks(int N, int causal, int window, int n_sink);
  * device.  Every wait inside the kernel is bounded (about attn_watchdog_ns
  * nanoseconds); a CTA whose wait expires drains its own in-flight copies and
  * tensor-core work, releases its tensor memory, records
- * ATTN_ERR_DEVICE_TIMEOUT here and returns.  Synchronises the device.
+ * ATTN_ERR_DEVICE_TIMEOUT here and returns.  The backward kernel also records
+ * ATTN_ERR_CUDA, and returns before doing any work, if the dynamic shared
+ * memory it was given cannot hold its 1024-byte aligned layout (a launch
+ * configuration fault; its outputs are then not written).  Synchronises the
+ * device.
  */
 int attn_get_status(void);
 
