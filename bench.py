@@ -560,10 +560,11 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args)
-    if args.decode:
-        return decode_bench(args)
-    if args.backward:
-        return backward_bench(args)
+    if args.decode or args.backward:
+        # single-GPU extra lines: under torchrun only rank 0 runs them
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        return decode_bench(args) if args.decode else backward_bench(args)
 
     import torch
     import exact_tiled_attention_44_b200 as A
