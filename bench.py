@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -53,10 +54,23 @@ KERNEL_SOURCES = ["exact_tiled_attention_44_b200/csrc/attn_kernel.cuh",
 BWD_KERNEL_SOURCES = ["exact_tiled_attention_44_b200/csrc/bwd_kernel.cuh"] + KERNEL_SOURCES
 
 
+def _code_only(text: str) -> str:
+    """Source without /* */ blocks, // comments, trailing blanks and empty lines
+    (none of the kernel files has // inside a string literal), so that editing a
+    comment does not count as a kernel change."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        line = line.split("//", 1)[0].rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
     for f in (sources or KERNEL_SOURCES):
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, f)).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,8 +14,8 @@
 // V_j in shared memory and dK_j, dV_j in tensor memory, and walks every query
 // tile i (of every query head that reads this K/V head) that keeps a pair
 // with tile j.  dK and dV are therefore owned by one CTA and written once;
-// dQ_i gets one 128 x d contribution per key tile, added to an fp32 buffer
-// with vector atomics.
+// dQ_i gets one 128 x d contribution per key tile, added to an fp32 buffer by
+// TMA bulk reductions (coalesced vector atomics for d < 64).
 //
 // Per step (query head h, query tile i), all products 128 x 128 (x d):
 //   MMA warp  S^T  = K_j Q_i^T           TMEM X (keys on lanes, queries on columns)
@@ -25,7 +25,7 @@
 //   compute   dS^T = P^T (dP^T - D) scale   16-bit over Y, and into shared memory
 //   MMA warp  dK  += dS^T Q_i            (A from TMEM)
 //             dQ   = dS K_j              (A = dS from shared memory, MN-major)
-//   compute   dQ rows (queries on lanes) -> fp32 atomics into the dQ buffer
+//   compute   dQ rows (queries on lanes) -> bulk reductions into the fp32 dQ buffer
 //
 // CTA (384 threads): warps 0-7 compute (two warpgroups; warpgroup w takes query columns
 // [64 w, 64 w + 64) of each tile and output columns [w d/2, (w+1) d/2)),
