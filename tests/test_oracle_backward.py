@@ -250,3 +250,27 @@ def test_tiled_recomputation_equals_the_definition(bs):
                                              causal, w, ns, slope, bs=bs)
             for a, b in zip(got, want):
                 assert np.abs(a - b).max() < 1e-12 * max(1.0, np.abs(b).max())
+
+
+def test_random_configurations_against_autograd():
+    """Random shapes, group sizes, masks, scales (any sign) and slopes: the
+    oracle's gradients equal torch autograd of the definition."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(st.integers(1, 2), st.sampled_from([(1, 1), (2, 1), (4, 2), (3, 3), (6, 2)]),
+           st.integers(1, 23), st.sampled_from([2, 4, 8]), st.booleans(),
+           st.integers(0, 6), st.integers(0, 3), st.booleans(),
+           st.floats(-1.5, 1.5, allow_nan=False), st.integers(0, 10_000))
+    def check(B, heads, N, d, causal, window, n_sink, alibi, scale, seed):
+        H, H_kv = heads
+        if window and not causal:
+            window = 0
+        q, k, v, do = _inputs(B, H, H_kv, N, d, seed)
+        sl = _slopes(H, alibi)
+        got = oracle.attention_backward(q, k, v, do, scale, causal, window, n_sink, sl)
+        ref = _torch_grads(q, k, v, do, scale, causal, window, n_sink, sl)
+        for a, b in zip(got, ref):
+            assert np.abs(a - b).max() <= 1e-10 * max(1.0, np.abs(b).max())
+
+    check()
