@@ -1,12 +1,15 @@
-"""Exact tiled attention forward for B200 (sm_100a): Python binding of libattn.so.
+"""Exact tiled attention for B200 (sm_100a): Python binding of libattn.so.
 
-Argument marshalling only.  Every arithmetic step of the forward runs in the
-CUDA kernel behind the C ABI declared in ``include/attn.h``; PyTorch supplies
-device memory and streams.  There is no CPU fallback: if the library is not
-built, or the device is not an sm_100 GPU, the calls raise.
+Argument marshalling only.  Every arithmetic step of the forward, the backward
+and the decoding step runs in the CUDA kernels behind the C ABI declared in
+``include/attn.h``; PyTorch supplies device memory and streams.  There is no
+CPU fallback: if the library is not built, or the device is not an sm_100 GPU,
+the calls raise.
 
-    from exact_tiled_attention_44_b200 import attention
-    o, lse = attention(q, k, v, causal=True)          # q,k,v: CUDA bf16/fp16 [B,H,N,d]
+    import exact_tiled_attention_44_b200 as A
+    o, lse = A.attention(q, k, v, causal=True)        # q,k,v: CUDA bf16/fp16 [B,H,N,d]
+    dq, dk, dv = A.attention_backward(q, k, v, o, do, lse, causal=True)
+    o_new, lse_new = A.decode(q_new, k_cache, v_cache)
 """
 from __future__ import annotations
 
