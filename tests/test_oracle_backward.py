@@ -135,7 +135,27 @@ def pin_closed_forms(impl):
         assert np.abs(dV[0, 0] - want).max() < 1e-12
 
 
-PINS = [pin_finite_differences, pin_torch_autograd, pin_invariants, pin_closed_forms]
+def pin_two_keys_by_hand(impl):
+    """One query q = 1 and two keys k = (0, ln 3), values v = (1, 5), scale 1,
+    dO = 1, no mask: P = (1/4, 3/4), O = 4, so dV = P = (1/4, 3/4),
+    dS_j = P_j (v_j - O) = (-3/4, 3/4), dK_j = dS_j q = (-3/4, 3/4) and
+    dQ = sum_j dS_j k_j = P_1 P_2 (v_1 - v_2)(k_1 - k_2) = (3/4) ln 3, worked out
+    by hand.  Posed as a 2-row non-causal problem whose second row has q = 0
+    and dO = 0, so that it adds nothing to dK and dV and its dQ is 0."""
+    import math
+    q = np.array([[[[1.0], [0.0]]]])
+    k = np.array([[[[0.0], [math.log(3.0)]]]])
+    v = np.array([[[[1.0], [5.0]]]])
+    do = np.array([[[[1.0], [0.0]]]])
+    dQ, dK, dV = impl(q, k, v, do, 1.0, False, 0, 0, None)
+    assert abs(dQ[0, 0, 0, 0] - 0.75 * math.log(3.0)) < 1e-14
+    assert abs(dQ[0, 0, 1, 0]) < 1e-14
+    assert np.abs(dK[0, 0, :, 0] - np.array([-0.75, 0.75])).max() < 1e-14
+    assert np.abs(dV[0, 0, :, 0] - np.array([0.25, 0.75])).max() < 1e-14
+
+
+PINS = [pin_finite_differences, pin_torch_autograd, pin_invariants, pin_closed_forms,
+        pin_two_keys_by_hand]
 
 
 def _oracle_impl(Q, K, V, dO, scale, causal, window, n_sink, slopes):
