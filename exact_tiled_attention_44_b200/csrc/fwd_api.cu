@@ -1,0 +1,88 @@
+// fwd_api.cu -- the forward's entry points attn_fwd and attn_fwd_alibi, and
+// the head dims 16, 32 and 64 (d = 128 is in fwd_d128.cu).
+#include "fwd_launch.cuh"
+
+namespace attn_host {
+
+// attn_fwd with an optional slope array (NULL: no position bias).
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+             const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
+             int n_sink, float scale, int dtype, void* stream) {
+  Sizes sz;
+  bool empty = false;
+  int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype, &sz,
+                    &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+
+  const bool bf16 = (dtype & 0xF) == ATTN_BF16;
+  const bool f32 = (dtype & ATTN_OUT_F32) != 0;
+  alignas(64) CUtensorMap mq, mk, mv;
+  if (encode_map(&mq, q, bf16, d, N, B * H) != ATTN_OK ||
+      encode_map(&mk, k, bf16, d, N, B * H_kv) != ATTN_OK ||
+      encode_map(&mv, v, bf16, d, N, B * H_kv) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+
+  attn::KernelParams kp;
+  kp.o = o;
+  kp.lse = lse;
+  kp.status = st->status;
+  kp.watchdog_ns = g_watchdog_ns.load(std::memory_order_relaxed);
+  kp.B = B;
+  kp.H = H;
+  kp.H_kv = H_kv;
+  kp.N = N;
+  kp.causal = causal;
+  // A window at least as long as the sequence keeps every causal key.
+  kp.window = (window >= N) ? 0 : window;
+  kp.n_sink = kp.window > 0 ? (n_sink < N ? n_sink : N) : 0;
+  kp.scale_log2 = scale * 1.4426950408889634f;
+  kp.n_qpairs = (N + 2 * attn::BM - 1) / (2 * attn::BM);
+  kp.n_kblocks = (N + attn::BN - 1) / attn::BN;
+  kp.num_units = B * H * kp.n_qpairs;
+  kp.alibi = slopes;
+  kp.withhold_loads = take_withhold();
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 16: return launch_d<16>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 32: return launch_d<32>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 64: return launch_d<64>(st, bf16, f32, mq, mk, mv, kp, s);
+    case 128: return launch_fwd_d128(st, bf16, f32, mq, mk, mv, kp, s);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace attn_host
+
+using namespace attn_host;
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int H_kv, int N, int d, int causal, int window, int n_sink, float scale, int dtype,
+             void* stream) {
+  return fwd_impl(q, k, v, o, lse, nullptr, B, H, H_kv, N, d, causal, window, n_sink, scale,
+                  dtype, stream);
+}
+
+int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const float* slopes, int B, int H, int H_kv, int N, int d, int causal,
+                   int window, int n_sink, float scale, int dtype, void* stream) {
+  Sizes sz;
+  bool empty = false;
+  const int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                          &sz, &empty);
+  if (rc != ATTN_OK || empty) return rc;
+  if (slopes == nullptr) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(slopes) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  if (overlaps(slopes, static_cast<size_t>(H) * sizeof(float), o, sz.o_bytes) ||
+      (lse != nullptr && overlaps(slopes, static_cast<size_t>(H) * sizeof(float), lse, sz.lse_bytes)))
+    return ATTN_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, slopes, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
+                  stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// host.h -- host-side pieces shared by the translation units of libattn.so:
+// per-device state, argument checks, TMA descriptor encoding and the process
+// wide counters.  Internal to the library (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+
+namespace attn_host {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  int* status = nullptr;           // device address of the status word
+  uint32_t attr_set = 0;           // one bit per forward kernel instantiation
+  uint32_t dec_attr_set = 0;       // one bit per decode kernel instantiation
+  uint32_t dec_small_attr_set = 0; // one bit per small-group decode kernel instantiation
+  uint32_t bwd_attr_set = 0;       // one bit per backward kernel instantiation
+};
+
+// Guards DeviceState initialisation and the per-kernel attribute bits.
+extern std::mutex g_mu;
+extern std::atomic<unsigned long long> g_watchdog_ns;
+extern std::atomic<unsigned long long> g_launches;
+extern std::atomic<int> g_withhold;     // launches left that withhold their loads (test hook)
+extern PFN_cuTensorMapEncodeTiled_v12000 g_encode;
+
+inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Sizes {
+  size_t q_bytes, kv_bytes, o_bytes, lse_bytes;
+  int elem, d;
+};
+
+// Pure argument validation of the forward's arguments: touches no CUDA API,
+// so it can be tested on a machine without a GPU.  Returns ATTN_OK and fills
+// `sz` when the call is well formed; `*empty` is set when there is nothing to
+// compute.
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
+             float scale, int dtype, Sizes* sz, bool* empty);
+
+// State of the current device, initialised on first use (an sm_100 device is
+// required; anything else is ATTN_ERR_UNSUPPORTED).
+int device_state(DeviceState** out);
+
+// 3-D view [z][rows][d] of a contiguous [.., n, d] 16-bit tensor; box =
+// (min(d, 64), 128, 1) with the swizzle span equal to the box's row bytes.
+int encode_map(CUtensorMap* map, const void* base, bool bf16, int d, int n, int z);
+
+// Takes one launch from the withhold-loads test hook, if any is pending.
+int take_withhold();
+
+// attn_fwd with an optional slope array (NULL: no position bias).
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+             const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
+             int n_sink, float scale, int dtype, void* stream);
+
+}  // namespace attn_host
