@@ -647,7 +647,9 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
     for (int idx = 0; idx < U.n_iter; ++idx) {
       const int j = block_at(U, idx);
       if (!tile_uses(U, t, j)) continue;
-      ok = wait_or_abort(bars + 8 * (B_S_FULL + t), s_ph, abort_flag, p);
+      // one verdict for the whole warp: the TMEM load and the vote below are
+      // warp-collective, so no lane may leave the loop alone
+      ok = warp_wait(bars + 8 * (B_S_FULL + t), s_ph, abort_flag, p);
       if (!ok) break;
       s_ph ^= 1u;
       tc_fence_after_sync();
@@ -783,7 +785,7 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
     }
     if (!ok) break;
     // epilogue: O = O_acc / l, written once; LSE = (m + log2 l) ln 2
-    ok = wait_or_abort(bars + 8 * (B_O_FULL + t), o_ph, abort_flag, p);
+    ok = warp_wait(bars + 8 * (B_O_FULL + t), o_ph, abort_flag, p);
     if (!ok) break;
     o_ph ^= 1u;
     tc_fence_after_sync();

@@ -66,6 +66,7 @@ struct BwdParams {
   int num_units;       // B * H_kv * ceil(n_tiles / 2) pair units
   const float* alibi;  // ALiBi slope per query head, or nullptr
   int smem_alloc;      // dynamic shared memory bytes given at launch
+  int withhold_loads;  // test hook: the copy warp issues nothing, so every wait runs out
 };
 
 template <int D>
@@ -328,6 +329,9 @@ __device__ void bw_tma_role(const BwdParams& p, const CUtensorMap* tmQ, const CU
                             uint32_t sbase, uint32_t bars, int lane, volatile int* abort_flag) {
   using G = Geo<D>;
   using W = BwGeo<D>;
+  // Failure-detection test: no copy is issued, so the other roles' bounded
+  // waits expire and the CTA reports ATTN_ERR_DEVICE_TIMEOUT and exits.
+  if (p.withhold_loads) return;
   uint32_t st_it = 0;
   int ul = 0;
   int kv_last = -1, qd_last[2] = {-1, -1};
@@ -545,9 +549,9 @@ __device__ void bw_compute_role(const BwdParams& p, const CUtensorMap* tmDQ, uin
       const bool masked = bw_needs_mask(p, q0, k0);
       const uint32_t nl = sbase + W::ST_OFF + s * W::ST_BYTES + 4 * 64 * wg;   // -LSE log2(e)
       const uint32_t dd = nl + 4 * 128;                                        // -scale D
-      ok = bw_wait(bars + 8 * (W_QD_FULL + s), ph, abort_flag, p);
+      ok = bw_warp_wait(bars + 8 * (W_QD_FULL + s), ph, abort_flag, p);
       if (!ok) break;
-      ok = bw_wait(bars + 8 * W_S_FULL, s_ph, abort_flag, p);
+      ok = bw_warp_wait(bars + 8 * W_S_FULL, s_ph, abort_flag, p);
       if (!ok) break;
       s_ph ^= 1u;
       tc_fence_after_sync();
@@ -594,7 +598,7 @@ __device__ void bw_compute_role(const BwdParams& p, const CUtensorMap* tmDQ, uin
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * W_P_FULL);
 
-      ok = bw_wait(bars + 8 * W_DP_FULL, dp_ph, abort_flag, p);
+      ok = bw_warp_wait(bars + 8 * W_DP_FULL, dp_ph, abort_flag, p);
       if (!ok) break;
       dp_ph ^= 1u;
       tc_fence_after_sync();
@@ -638,7 +642,7 @@ __device__ void bw_compute_role(const BwdParams& p, const CUtensorMap* tmDQ, uin
       }
 
       // dQ rows: lane t now holds query q0 + t
-      ok = bw_wait(bars + 8 * W_DQ_FULL, dq_ph, abort_flag, p);
+      ok = bw_warp_wait(bars + 8 * W_DQ_FULL, dq_ph, abort_flag, p);
       if (!ok) break;
       dq_ph ^= 1u;
       tc_fence_after_sync();
@@ -709,7 +713,7 @@ __device__ void bw_compute_role(const BwdParams& p, const CUtensorMap* tmDQ, uin
     }
     if (!ok) break;
     // epilogue: dV and dK rows of key kt
-    ok = bw_wait(bars + 8 * W_ACC_FULL, acc_ph, abort_flag, p);
+    ok = bw_warp_wait(bars + 8 * W_ACC_FULL, acc_ph, abort_flag, p);
     if (!ok) break;
     acc_ph ^= 1u;
     tc_fence_after_sync();

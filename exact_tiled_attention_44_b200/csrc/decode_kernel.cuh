@@ -52,6 +52,7 @@ struct DecodeParams {
   float scale_log2;   // scale * log2(e)
   int n_splits;       // split s covers keys [s * split_keys, min(N_kv, (s + 1) * split_keys))
   int split_keys;     // a multiple of DEC_T
+  int withhold_loads; // test hook: no tile is loaded, so every wait on a tile runs out
 };
 
 template <int D>
@@ -166,6 +167,8 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   bool ok = true;
   int issued_last[2] = {-1, -1};        // parity of the last load into each stage (warp 0)
   auto issue = [&](int j0, int n) {
+    // failure-detection test: nothing is loaded (and nothing is left to drain)
+    if (p.withhold_loads) return true;
     const int st = n & 1;
     const uint32_t ph = (static_cast<uint32_t>(n) >> 1) & 1u;
     if (!mbar_try_wait(bars + 8 * (DB_EMPTY + st), ph ^ 1u) &&
@@ -503,6 +506,8 @@ attn_decode_small_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
   for (int s = 0; s < NS; ++s) issued_last[s] = -1;
   auto issue = [&](int j0, int n) {
+    // failure-detection test: nothing is loaded (and nothing is left to drain)
+    if (p.withhold_loads) return true;
     const int st = n % NS;
     const uint32_t ph = static_cast<uint32_t>(n / NS) & 1u;
     const uint32_t empty = bars + 8 * (NS + st);
