@@ -25,7 +25,7 @@ __all__ = [
     "attn_decode_noalloc_raw", "attention_backward", "attn_bwd_raw", "bwd_workspace_bytes",
     "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
-    "error_string",
+    "test_count_blocks", "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
     "ATTN_BF16", "ATTN_FP16", "ATTN_OUT_F32",
@@ -45,7 +45,8 @@ EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_s
                     "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
-                    "attn_test_withhold_loads", "attn_bwd", "attn_bwd_workspace_bytes")
+                    "attn_test_withhold_loads", "attn_test_count_blocks", "attn_bwd",
+                    "attn_bwd_workspace_bytes")
 
 _LIB = None
 
@@ -98,6 +99,8 @@ def load_library():
     lib.attn_launch_count.restype = ctypes.c_ulonglong
     lib.attn_test_withhold_loads.argtypes = [ci]
     lib.attn_test_withhold_loads.restype = ci
+    lib.attn_test_count_blocks.argtypes = [vp]
+    lib.attn_test_count_blocks.restype = ci
     lib.attn_bwd.argtypes = [vp] * 11 + [ctypes.c_longlong] + [ci] * 8 + [cf, ci, vp]
     lib.attn_bwd.restype = ci
     lib.attn_bwd_workspace_bytes.argtypes = [ci] * 5
@@ -137,6 +140,19 @@ def test_withhold_loads(n_launches: int) -> int:
     """Failure-detection hook: the next n launches issue no copies, so their
     waits run into the watchdog (see include/attn.h)."""
     return int(load_library().attn_test_withhold_loads(int(n_launches)))
+
+
+def test_count_blocks(counter: torch.Tensor | None) -> int:
+    """Schedule test hook: while set, forward and backward launches add the
+    score tiles (forward) or steps (backward) they compute to ``counter``, a
+    one-element int64 CUDA tensor the caller zeroes; None turns it off (see
+    include/attn.h)."""
+    if counter is None:
+        return int(load_library().attn_test_count_blocks(None))
+    if (not counter.is_cuda or counter.dtype != torch.int64 or counter.numel() != 1
+            or not counter.is_contiguous()):
+        raise ValueError("counter must be a one-element contiguous int64 CUDA tensor")
+    return int(load_library().attn_test_count_blocks(counter.data_ptr()))
 
 
 def alibi_slopes(H: int, device=None) -> torch.Tensor:

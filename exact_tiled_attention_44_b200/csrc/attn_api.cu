@@ -24,6 +24,7 @@ std::mutex g_mu;
 std::atomic<unsigned long long> g_watchdog_ns{2000000000ull};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<int> g_withhold{0};
+std::atomic<unsigned long long*> g_block_count{nullptr};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -250,6 +251,11 @@ unsigned long long attn_set_watchdog_ns(unsigned long long ns) {
 int attn_test_withhold_loads(int n_launches) {
   if (n_launches < 0) return ATTN_ERR_INVALID_ARG;
   g_withhold.store(n_launches);
+  return ATTN_OK;
+}
+
+int attn_test_count_blocks(unsigned long long* counter) {
+  g_block_count.store(counter);
   return ATTN_OK;
 }
 

@@ -75,6 +75,7 @@ struct KernelParams {
   int num_units;      // B * H * n_qpairs
   const float* alibi; // ALiBi slope per query head ([H], device), used by the ALIBI kernels
   int withhold_loads; // test hook: the TMA warp issues nothing, so every wait runs out
+  unsigned long long* block_count;  // test hook: S tiles computed are added here (or nullptr)
 };
 
 // Shared-memory geometry for head dimension D (16-bit elements).  A 128 x D
@@ -455,6 +456,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
                          volatile int* abort_flag) {
   uint32_t kv_it = 0, p_ph[2] = {0, 0};
   uint32_t q_uses[Q_SLOTS] = {0, 0, 0};
+  unsigned long long n_s = 0;   // (Q tile, K/V block) score tiles issued, for the test hook
   bool ok = true;
   const int rounds = num_rounds(gridDim.x, p.num_units);
   int ul = 0;
@@ -503,6 +505,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
           mma_commit(bars + 8 * (B_S_FULL + t));
         }
         __syncwarp();
+        ++n_s;
       }
       if (!ok) break;
       if (elect_one()) {
@@ -550,6 +553,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
             mma_commit(bars + 8 * (B_S_FULL + 0));
           }
           __syncwarp();
+          ++n_s;
         }
       }
       // Q tile 1: P1 V_j, then S1 for the next block
@@ -585,6 +589,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         }
       }
       __syncwarp();
+      if (has_next && tile_uses(U, 1, jn)) ++n_s;
       // Once Q tile 0 has no block left in this unit (its last P_0 V is
       // issued and no S_0 follows), its next S is the next unit's first one:
       // issue it now, so that softmax 0 finds it ready after its epilogue
@@ -606,12 +611,17 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
             mma_commit(bars + 8 * (B_S_FULL + 0));
           }
           __syncwarp();
+          ++n_s;
           s0_pre = true;
         }
       }
     }
     kv_it += U.n_iter;
     ++ul;
+  }
+  if (p.block_count != nullptr) {
+    if (elect_one()) atomicAdd(p.block_count, n_s);
+    __syncwarp();
   }
   // Every MMA this warp issued has completed once the drain barrier flips.
   if (elect_one()) mma_commit(bars + 8 * B_DRAIN);

@@ -184,6 +184,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   bp.num_units = static_cast<int>(units);
   bp.alibi = slopes;
   bp.withhold_loads = take_withhold();
+  bp.block_count = g_block_count.load();
   const long long rows = static_cast<long long>(B) * H * N;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool al = slopes != nullptr;

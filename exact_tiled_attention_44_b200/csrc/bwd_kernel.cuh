@@ -67,6 +67,7 @@ struct BwdParams {
   const float* alibi;  // ALiBi slope per query head, or nullptr
   int smem_alloc;      // dynamic shared memory bytes given at launch
   int withhold_loads;  // test hook: the copy warp issues nothing, so every wait runs out
+  unsigned long long* block_count;  // test hook: (key tile, query tile) steps are added here
 };
 
 template <int D>
@@ -414,6 +415,7 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
   using G = Geo<D>;
   using W = BwGeo<D>;
   uint32_t st_it = 0, p_ph = 0, ds_ph = 0, dqf_ph = 0, accf_ph = 0;
+  unsigned long long n_steps = 0;   // steps issued, for the test hook
   bool any_dq = false;
   bool ok = true;
   int ul = 0;
@@ -477,6 +479,7 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
       }
       __syncwarp();
       any_dq = true;
+      ++n_steps;
     }
     if (!ok) break;
     if (elect_one()) {
@@ -485,6 +488,10 @@ __device__ void bw_mma_role(const BwdParams& p, uint32_t tmem, uint32_t sbase, u
     }
     __syncwarp();
     ++ul;
+  }
+  if (p.block_count != nullptr) {
+    if (elect_one()) atomicAdd(p.block_count, n_steps);
+    __syncwarp();
   }
   if (elect_one()) mma_commit(bars + 8 * W_DRAIN);
   __syncwarp();

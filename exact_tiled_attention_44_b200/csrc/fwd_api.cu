@@ -44,6 +44,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
   kp.num_units = B * H * kp.n_qpairs;
   kp.alibi = slopes;
   kp.withhold_loads = take_withhold();
+  kp.block_count = g_block_count.load();
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {

@@ -34,6 +34,7 @@ extern std::mutex g_mu;
 extern std::atomic<unsigned long long> g_watchdog_ns;
 extern std::atomic<unsigned long long> g_launches;
 extern std::atomic<int> g_withhold;     // launches left that withhold their loads (test hook)
+extern std::atomic<unsigned long long*> g_block_count;   // block-count test hook (or nullptr)
 extern PFN_cuTensorMapEncodeTiled_v12000 g_encode;
 
 inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

@@ -288,6 +288,21 @@ unsigned long long attn_launch_count(void);
  */
 int attn_test_withhold_loads(int n_launches);
 
+/*
+ * attn_test_count_blocks -- schedule test hook (the paper has no counterpart).
+ * While `counter` is non-NULL, every later attn_fwd / attn_fwd_alibi launch
+ * adds to the device uint64 at `counter` the number of (128-row query tile,
+ * 128-key block) score tiles it computed, and every attn_bwd launch the
+ * number of (key tile, query tile) steps of its tiled kernel, with one atomic
+ * add per CTA.  A test compares the sum with attn_visited_blocks() times
+ * B * H ("Tiled attention with online softmax", exercise 3: count the block
+ * pairs the tiled loop visits).  `counter` is caller-owned device memory,
+ * 8-byte aligned, zeroed by the caller; NULL turns the hook off (the default).
+ * Process-wide and not synchronised with launches in flight: set it between
+ * launches only.  Returns ATTN_OK.
+ */
+int attn_test_count_blocks(unsigned long long* counter);
+
 #ifdef __cplusplus
 }
 #endif

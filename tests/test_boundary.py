@@ -187,6 +187,12 @@ def test_withhold_hook_arguments():
     assert A.test_withhold_loads(0) == A.ATTN_OK
 
 
+def test_count_blocks_hook_arguments():
+    assert A.test_count_blocks(None) == A.ATTN_OK
+    with pytest.raises(ValueError):
+        A.test_count_blocks(torch.zeros(1, dtype=torch.int64))         # not on a GPU
+
+
 # ------------------------------------------------------------------ decode entry points
 
 
