@@ -40,6 +40,12 @@
  *     and watchdog expiries are reported by attn_get_status().
  *   - Results are deterministic: equal inputs give bitwise-equal outputs,
  *     except attn_bwd's dQ (see there).
+ *   - Per device, the first call records device addresses of the library's
+ *     own __device__ objects (its status word, the static scratch array of
+ *     attn_decode_noalloc) and keeps them for the life of the process.  The
+ *     library therefore does not support cudaDeviceReset (or any other loss
+ *     of the primary context) between calls: after one, those addresses may
+ *     be stale.
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -250,8 +256,9 @@ long long attn_unmasked_pairs(int N, int causal, int window, int n_sink);
  * attn_visited_blocks -- host only: the number of (128-query-row block,
  * 128-key block) pairs the kernel's schedule computes for one head (the same
  * set for the forward and for attn_bwd).  A block
- * pair is visited iff it holds at least one kept pair (causal, window and sink
- * skipping as in Lab 3's "only key blocks at or before this query block").
+ * pair is visited iff it holds at least one kept pair (this generalises the
+ * causal block skipping of "Tiled attention with online softmax", Lab 3, to
+ * windows and sinks).
  * Returns -1 for invalid arguments.
  */
 long long attn_visited_blocks(int N, int causal, int window, int n_sink);
