@@ -114,7 +114,8 @@ enum BarSlot : int {
   B_P_FULL = B_S_FULL + 2,             // [2]
   B_O_FULL = B_P_FULL + 2,             // [2]
   B_DRAIN = B_O_FULL + 2,
-  B_COUNT = B_DRAIN + 1
+  B_EPI = B_DRAIN + 1,                 // [2] a tile's output rows are staged in shared memory
+  B_COUNT = B_EPI + 2
 };
 constexpr int TMEM_SLOT_OFF = 8 * B_COUNT;
 constexpr int ABORT_FLAG_OFF = TMEM_SLOT_OFF + 4;
@@ -366,7 +367,12 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     const Unit U = decode_unit(u, p);
-    // Q tile 0 first: its slot was released by the unit before last.
+    // Loads in the order their ring stages and Q slots are released, so
+    // that no load waits behind one whose slot frees later: Q tile 0 (its
+    // slot was released by the unit before last), the first K block (whose
+    // stage the unit before released one block before its end: the early
+    // S_0 of this unit needs it), the first V block, then Q tile 1 (its slot
+    // frees only when the unit before has issued its last S MMAs).
     ok = load_q(U, ul, 0);
     if (!ok) break;
     const int kvz = U.b * p.H_kv + U.g;
@@ -384,12 +390,6 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       }
       __syncwarp();
       k_last[s] = ph;
-      // Q tile 1 after the first K tile: its slot is the previous unit's
-      // tile-0 slot, free once that unit's last S MMAs are done.
-      if (idx == 0 && U.n_active > 1) {
-        ok = load_q(U, ul, 1);
-        if (!ok) break;
-      }
       ok = warp_wait(bars + 8 * (B_V_EMPTY + s), ph ^ 1u, abort_flag, p);
       if (!ok) break;
       if (elect_one()) {
@@ -400,6 +400,10 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       }
       __syncwarp();
       v_last[s] = ph;
+      if (idx == 0 && U.n_active > 1) {
+        ok = load_q(U, ul, 1);
+        if (!ok) break;
+      }
     }
     ++ul;
   }
@@ -630,8 +634,9 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
 }
 
 template <int D, bool BF16, bool OUT_F32, bool ALIBI>
-__device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars, int t,
-                             int warp_in_wg, int lane, volatile int* abort_flag) {
+__device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint32_t tmem,
+                             uint32_t sbase, uint32_t bars, int t, int warp_in_wg, int lane,
+                             volatile int* abort_flag) {
   using G = Geo<D>;
   constexpr int OC = D >= 32 ? 32 : 16;   // TMEM columns per O load/store
   const int row_in_tile = warp_in_wg * 32 + lane;
@@ -639,12 +644,28 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
   const uint32_t s_tmem = tmem + lane_base + G::S_COL0 + t * BN;
   const uint32_t o_tmem = tmem + lane_base + G::O_COL0 + t * D;
   const float c = p.scale_log2;
-  uint32_t s_ph = 0, o_ph = 0;
+  // 16-bit output rows of 128 bytes per 64-column chunk are staged in shared
+  // memory and written by TMA; other outputs are stored from registers.
+  constexpr bool STAGED = !OUT_F32 && G::CB == 128;
+  uint32_t s_ph = 0, o_ph = 0, epi_ph = 0;
   bool ok = true;
+  int ul = -1;
+  // Q_EMPTY barrier of the slot whose staged output a TMA store issued by
+  // this thread (warp 0, lane 0) may still be reading, or 0.  The wait is
+  // deferred to the next S wait, where the warp would idle anyway.
+  uint32_t staged_slot = 0;
+  auto release_stage = [&]() {
+    if (STAGED && staged_slot != 0) {
+      bulk_wait_group_read0();
+      mbar_arrive(staged_slot);
+      staged_slot = 0;
+    }
+  };
   const int rounds = num_rounds(gridDim.x, p.num_units);
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
+    ++ul;
     const Unit U = decode_unit(u, p);
     if (t >= U.n_active) continue;
     const int r0 = U.q0 + t * BM;
@@ -657,6 +678,7 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
     for (int idx = 0; idx < U.n_iter; ++idx) {
       const int j = block_at(U, idx);
       if (!tile_uses(U, t, j)) continue;
+      release_stage();
       // one verdict for the whole warp: the TMEM load and the vote below are
       // warp-collective, so no lane may leave the loop alone
       ok = warp_wait(bars + 8 * (B_S_FULL + t), s_ph, abort_flag, p);
@@ -668,7 +690,9 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
       const int c0 = j * BN;
       const bool masked = block_needs_mask(p, r0, c0);
       float m_blk;
-      if (masked || ALIBI) {
+      // Logits already scaled (and biased) in sr, instead of raw scores.
+      const bool prescaled = ALIBI || (masked && c == 0.f);
+      if (prescaled) {
         // Scale first (adding the position bias -slope |i - j|), then drop
         // masked keys with -inf (any sign of scale).  Kept keys of this row,
         // in block-local columns e = j - c0:
@@ -712,6 +736,36 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
         }
         m_blk = fmaxf(m0, m1);
       } else {
+        if (masked) {
+          // A masked key gets the raw score -inf (+inf for a negative scale),
+          // which the scale turns into -inf; the raw extreme and the exps
+          // below then run as for an interior block.  Kept keys of this row,
+          // in block-local columns e = j - c0:
+          //   e <= hi (causal limit and key padding) and (e >= lo (window) or e < sk (sinks)).
+          // The block's geometry says which of the bounds can bite (the same
+          // for every row), so most blocks test one or two of them.
+          const uint32_t gone = c > 0.f ? 0xff800000u : 0x7f800000u;
+          const int hi = (p.causal ? min(row, p.N - 1) : p.N - 1) - c0;
+          const int lo = row - p.window + 1 - c0;
+          const int sk = p.n_sink - c0;
+          const bool win_in = p.window > 0 && r0 + BM - p.window > c0;          // a window starts inside
+          const bool win_after = p.window > 0 && r0 - p.window + 1 - c0 >= BN;  // every window starts after
+          const bool hi_in = c0 + BN > p.N || (p.causal && c0 + BN - 1 > r0);   // a causal / padding edge
+          if (win_after && !hi_in) {
+            // before every row's window: only the sinks are kept
+#pragma unroll
+            for (int e = 0; e < 128; ++e) sr[e] = (e < sk) ? sr[e] : gone;
+          } else if (!win_in && !win_after) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) sr[e] = (e <= hi) ? sr[e] : gone;
+          } else if (win_in && !hi_in && sk <= 0) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) sr[e] = (e >= lo) ? sr[e] : gone;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) sr[e] = ((e <= hi) && (e >= lo || e < sk)) ? sr[e] : gone;
+          }
+        }
         // raw-score extreme, then one multiply: max of s*c is c*max(s) for c >= 0
         // and c*min(s) for c < 0
         float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
@@ -742,7 +796,7 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
         m_run = m_new;
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 cc2 = (masked || ALIBI) ? make_float2(1.f, 1.f) : make_float2(c, c);
+      const float2 cc2 = prescaled ? make_float2(1.f, 1.f) : make_float2(c, c);
       const float2 nm2 = make_float2(-mref, -mref);
       // Two denominators: le sums the fp32 weights (for the LSE), lr sums the
       // same 16-bit-rounded weights the P V MMA consumes (for O, so that every
@@ -801,44 +855,98 @@ __device__ void softmax_role(const KernelParams& p, uint32_t tmem, uint32_t bars
     tc_fence_after_sync();
     const float inv_l = 1.f / l_round;
     const bool valid = row < p.N;
-    const size_t row_off = (static_cast<size_t>(U.bh) * p.N + row) * D;
+    const uint32_t q_empty = bars + 8 * (B_Q_EMPTY + q_slot(ul, t));
+    if constexpr (STAGED) {
+      // O / l as 16-bit rows in this tile's Q slot (no longer read: the O_FULL
+      // commit follows the tile's last S MMA), in the layout of the output's
+      // TMA box: 64-column chunks of 128 rows x 128 bytes, 128-byte swizzle.
+      // Warp 0 then writes the tile with TMA stores (rows >= N are clipped)
+      // and releases the slot once the stores have read it.
+      const uint32_t stage = sbase + G::Q_OFF + q_slot(ul, t) * G::TILE_BYTES;
+      const uint32_t row_addr = stage + row_in_tile * 128;
 #pragma unroll
-    for (int cc = 0; cc < D / OC; ++cc) {
-      uint32_t orr[OC];
-      tmem_ld_cols<OC>(o_tmem + cc * OC, orr);
-      if (valid) {
-        if constexpr (OUT_F32) {
-          float* dst = reinterpret_cast<float*>(p.o) + row_off + cc * OC;
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t orr[32];
+        tmem_ld_32x32b_x32(o_tmem + cc * 32, orr);
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < OC; e += 4) {
-            const float4 v4 = make_float4(
-                __uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l,
-                __uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
-            *reinterpret_cast<float4*>(dst + e) = v4;
-          }
-        } else {
-          uint32_t packed[OC / 2];
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
+                              __uint_as_float(orr[2 * e + 1]) * inv_l);
 #pragma unroll
-          for (int e = 0; e < OC / 2; ++e)
-            packed[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
-                                    __uint_as_float(orr[2 * e + 1]) * inv_l);
-          uint16_t* dst = reinterpret_cast<uint16_t*>(p.o) + row_off + cc * OC;
-#pragma unroll
-          for (int e = 0; e < OC / 2; e += 4)
-            *reinterpret_cast<uint4*>(dst + 2 * e) =
-                make_uint4(packed[e], packed[e + 1], packed[e + 2], packed[e + 3]);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int unit = (cc & 1) * 4 + k4;   // 16-byte unit within the 128-byte row
+          st_shared_v4(row_addr + (cc >> 1) * G::CHUNK_BYTES + ((unit ^ (row_in_tile & 7)) << 4),
+                       pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (B_EPI + t));
+      if (warp_in_wg == 0) {
+        ok = warp_wait(bars + 8 * (B_EPI + t), epi_ph, abort_flag, p);
+        if (ok && lane == 0) {
+#pragma unroll
+          for (int cch = 0; cch < G::NCH; ++cch)
+            tma_store_3d(tmO, stage + cch * G::CHUNK_BYTES, cch * G::CW, r0, U.bh);
+          bulk_commit_group();
+          // the slot is released once the store has read it (see release_stage)
+          staged_slot = q_empty;
+        }
+        __syncwarp();
+      }
+      epi_ph ^= 1u;
+    } else {
+      const size_t row_off = (static_cast<size_t>(U.bh) * p.N + row) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / OC; ++cc) {
+        uint32_t orr[OC];
+        tmem_ld_cols<OC>(o_tmem + cc * OC, orr);
+        if (valid) {
+          if constexpr (OUT_F32) {
+            float* dst = reinterpret_cast<float*>(p.o) + row_off + cc * OC;
+#pragma unroll
+            for (int e = 0; e < OC; e += 4) {
+              const float4 v4 = make_float4(
+                  __uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l,
+                  __uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
+              *reinterpret_cast<float4*>(dst + e) = v4;
+            }
+          } else {
+            uint32_t packed[OC / 2];
+#pragma unroll
+            for (int e = 0; e < OC / 2; ++e)
+              packed[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
+                                      __uint_as_float(orr[2 * e + 1]) * inv_l);
+            uint16_t* dst = reinterpret_cast<uint16_t*>(p.o) + row_off + cc * OC;
+#pragma unroll
+            for (int e = 0; e < OC / 2; e += 4)
+              *reinterpret_cast<uint4*>(dst + 2 * e) =
+                  make_uint4(packed[e], packed[e + 1], packed[e + 2], packed[e + 3]);
+          }
+        }
+      }
+      // the slot was not used for staging
+      if (warp_in_wg == 0 && lane == 0) mbar_arrive(q_empty);
     }
     if (valid && p.lse != nullptr)
       p.lse[static_cast<size_t>(U.bh) * p.N + row] = (m_run + __log2f(l_exact)) * 0.69314718055994531f;
+  }
+  // the output stores this warp issued complete before the CTA can exit
+  if (STAGED && warp_in_wg == 0) {
+    if (lane == 0) {
+      release_stage();
+      bulk_wait_group0();
+    }
+    __syncwarp();
   }
 }
 
 template <int D, bool BF16, bool OUT_F32, bool ALIBI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const KernelParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const KernelParams p) {
   using G = Geo<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment keeps every tile on a swizzle-pattern boundary.
@@ -855,7 +963,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < Q_SLOTS; ++s) {
       mbar_init(bars + 8 * (B_Q_FULL + s), 1);
-      mbar_init(bars + 8 * (B_Q_EMPTY + s), 1);
+      // the last S MMA that reads the slot, and the epilogue that stages the
+      // tile's output in it afterwards
+      mbar_init(bars + 8 * (B_Q_EMPTY + s), 2);
     }
     for (int s = 0; s < NUM_STAGES; ++s) {
       mbar_init(bars + 8 * (B_K_FULL + s), 1);
@@ -869,6 +979,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(bars + 8 * (B_O_FULL + t), 1);
     }
     mbar_init(bars + 8 * B_DRAIN, 1);
+    mbar_init(bars + 8 * (B_EPI + 0), 4);   // one arrival per softmax warp
+    mbar_init(bars + 8 * (B_EPI + 1), 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -880,6 +992,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (!OUT_F32) tma_prefetch_desc(&tmO);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -891,7 +1004,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // smaller one.
   if (warp < 8) {
     regs_increase<SOFTMAX_REGS>();
-    softmax_role<D, BF16, OUT_F32, ALIBI>(p, tmem, bars, warp / 4, warp % 4, lane, abort_flag);
+    softmax_role<D, BF16, OUT_F32, ALIBI>(p, &tmO, tmem, sbase, bars, warp / 4, warp % 4, lane,
+                                          abort_flag);
     tc_fence_before_sync();
     __syncthreads();
   } else {

@@ -19,10 +19,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
 
   const bool bf16 = (dtype & 0xF) == ATTN_BF16;
   const bool f32 = (dtype & ATTN_OUT_F32) != 0;
-  alignas(64) CUtensorMap mq, mk, mv;
+  alignas(64) CUtensorMap mq, mk, mv, mo;
   if (encode_map(&mq, q, bf16, d, N, B * H) != ATTN_OK ||
       encode_map(&mk, k, bf16, d, N, B * H_kv) != ATTN_OK ||
       encode_map(&mv, v, bf16, d, N, B * H_kv) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+  // the output's map (16-bit outputs are written by TMA stores; an fp32
+  // output is stored from registers and the map is not read)
+  if (f32)
+    mo = mq;
+  else if (encode_map(&mo, o, bf16, d, N, B * H) != ATTN_OK)
     return ATTN_ERR_CUDA;
 
   attn::KernelParams kp;
@@ -48,10 +54,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 16: return launch_d<16>(st, bf16, f32, mq, mk, mv, kp, s);
-    case 32: return launch_d<32>(st, bf16, f32, mq, mk, mv, kp, s);
-    case 64: return launch_d<64>(st, bf16, f32, mq, mk, mv, kp, s);
-    case 128: return launch_fwd_d128(st, bf16, f32, mq, mk, mv, kp, s);
+    case 16: return launch_d<16>(st, bf16, f32, mq, mk, mv, mo, kp, s);
+    case 32: return launch_d<32>(st, bf16, f32, mq, mk, mv, mo, kp, s);
+    case 64: return launch_d<64>(st, bf16, f32, mq, mk, mv, mo, kp, s);
+    case 128: return launch_fwd_d128(st, bf16, f32, mq, mk, mv, mo, kp, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }

@@ -9,7 +9,8 @@ namespace attn_host {
 
 template <int D, bool BF16, bool F32, bool ALIBI>
 int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
-               const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
+               const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
+               cudaStream_t stream) {
   auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI>;
   // At least half of the SM's shared memory, so that two CTAs can never share
   // an SM (each allocates all 512 TMEM columns).
@@ -29,33 +30,35 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
     }
   }
   const int grid = kp.num_units < st->sm_count ? kp.num_units : st->sm_count;
-  kern<<<grid, attn::NUM_THREADS, smem, stream>>>(mq, mk, mv, kp);
+  kern<<<grid, attn::NUM_THREADS, smem, stream>>>(mq, mk, mv, mo, kp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool ALIBI>
 int launch_da(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
-              const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
+              const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
+              cudaStream_t stream) {
   const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
   const int bit = dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
   if (bf16)
-    return f32 ? launch_one<D, true, true, ALIBI>(st, bit, mq, mk, mv, kp, stream)
-               : launch_one<D, true, false, ALIBI>(st, bit, mq, mk, mv, kp, stream);
-  return f32 ? launch_one<D, false, true, ALIBI>(st, bit, mq, mk, mv, kp, stream)
-             : launch_one<D, false, false, ALIBI>(st, bit, mq, mk, mv, kp, stream);
+    return f32 ? launch_one<D, true, true, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream)
+               : launch_one<D, true, false, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream);
+  return f32 ? launch_one<D, false, true, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream)
+             : launch_one<D, false, false, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream);
 }
 
 template <int D>
 int launch_d(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
-             const CUtensorMap& mv, const attn::KernelParams& kp, cudaStream_t stream) {
-  return kp.alibi != nullptr ? launch_da<D, true>(st, bf16, f32, mq, mk, mv, kp, stream)
-                             : launch_da<D, false>(st, bf16, f32, mq, mk, mv, kp, stream);
+             const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
+             cudaStream_t stream) {
+  return kp.alibi != nullptr ? launch_da<D, true>(st, bf16, f32, mq, mk, mv, mo, kp, stream)
+                             : launch_da<D, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
 }
 
 // The d = 128 instantiations (compiled in their own translation unit).
 int launch_fwd_d128(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq,
-                    const CUtensorMap& mk, const CUtensorMap& mv, const attn::KernelParams& kp,
-                    cudaStream_t stream);
+                    const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                    const attn::KernelParams& kp, cudaStream_t stream);
 
 }  // namespace attn_host
