@@ -25,6 +25,7 @@ std::atomic<unsigned long long> g_watchdog_ns{2000000000ull};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<int> g_withhold{0};
 std::atomic<unsigned long long*> g_block_count{nullptr};
+std::mutex g_host_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -157,18 +158,74 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(dq, q, sz.q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k, sz.kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v, sz.kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  rc = attn_fwd(dq, dk, dv, dout, dlse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype,
-                stream);
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
-  if (cudaMemcpyAsync(o, dout, sz.o_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool with_lse = lse != nullptr && dlse != nullptr;
+  // The problem is cut into chunks of consecutive (batch, K/V head) groups.
+  // A group's q, o and lse rows (its H / H_kv query heads) and its k, v rows
+  // are contiguous in every buffer, and a run of T groups is itself an
+  // attention problem of T batches of G query heads over one K/V head.  The
+  // host->device copies of chunk c+1 (copy stream 1), the forward of chunk c
+  // (the caller's stream) and the device->host copies of chunk c-1 (copy
+  // stream 2) overlap; events order them, and the caller's stream waits for
+  // the last copy, so the contract of a single stream holds.
+  const long long groups = static_cast<long long>(B) * H_kv;
+  const int G = H / H_kv;
+  // chunked LSE rows must keep the 16-byte alignment attn_fwd requires
+  const bool lse_ok = !with_lse || (static_cast<long long>(G) * N) % 4 == 0;
+  const int n_chunks = lse_ok ? static_cast<int>(groups < kHostChunks ? groups : kHostChunks) : 1;
+  const size_t q_grp = static_cast<size_t>(G) * N * d * sz.elem;
+  const size_t kv_grp = static_cast<size_t>(N) * d * sz.elem;
+  const size_t o_grp = sz.o_bytes / static_cast<size_t>(groups);
+  const size_t l_grp = static_cast<size_t>(G) * N * sizeof(float);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  if (!st->host_ready) {
+    if (cudaStreamCreateWithFlags(&st->copy_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st->copy_out, cudaStreamNonBlocking) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    for (int i = 0; i < 2 * kHostChunks + 2; ++i)
+      if (cudaEventCreateWithFlags(&st->ev[i], cudaEventDisableTiming) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    st->host_ready = true;
+  }
+  cudaEvent_t start = st->ev[2 * kHostChunks], done = st->ev[2 * kHostChunks + 1];
+  if (cudaEventRecord(start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(st->copy_in, start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(st->copy_out, start, 0) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  if (lse != nullptr && dlse != nullptr &&
-      cudaMemcpyAsync(lse, dlse, sz.lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  const auto at = [](const void* base, size_t off) {
+    return static_cast<const char*>(base) + off;
+  };
+  long long g0 = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    const long long g1 = groups * (c + 1) / n_chunks;
+    const size_t T = static_cast<size_t>(g1 - g0);
+    cudaEvent_t in = st->ev[2 * c], out = st->ev[2 * c + 1];
+    char* dqc = const_cast<char*>(at(dq, g0 * q_grp));
+    char* dkc = const_cast<char*>(at(dk, g0 * kv_grp));
+    char* dvc = const_cast<char*>(at(dv, g0 * kv_grp));
+    char* doc = const_cast<char*>(at(dout, g0 * o_grp));
+    float* dlc = with_lse ? reinterpret_cast<float*>(const_cast<char*>(at(dlse, g0 * l_grp))) : nullptr;
+    if (cudaMemcpyAsync(dqc, at(q, g0 * q_grp), T * q_grp, cudaMemcpyHostToDevice, st->copy_in) != cudaSuccess ||
+        cudaMemcpyAsync(dkc, at(k, g0 * kv_grp), T * kv_grp, cudaMemcpyHostToDevice, st->copy_in) != cudaSuccess ||
+        cudaMemcpyAsync(dvc, at(v, g0 * kv_grp), T * kv_grp, cudaMemcpyHostToDevice, st->copy_in) != cudaSuccess ||
+        cudaEventRecord(in, st->copy_in) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    rc = attn_fwd(dqc, dkc, dvc, doc, dlc, static_cast<int>(T), G, 1, N, d, causal, window, n_sink,
+                  scale, dtype, stream);
+    if (rc != ATTN_OK) return rc;
+    if (cudaEventRecord(out, s) != cudaSuccess || cudaStreamWaitEvent(st->copy_out, out, 0) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<char*>(at(o, g0 * o_grp)), doc, T * o_grp, cudaMemcpyDeviceToHost,
+                        st->copy_out) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (with_lse && cudaMemcpyAsync(const_cast<char*>(at(lse, g0 * l_grp)), dlc, T * l_grp,
+                                    cudaMemcpyDeviceToHost, st->copy_out) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    g0 = g1;
+  }
+  if (cudaEventRecord(done, st->copy_out) != cudaSuccess || cudaStreamWaitEvent(s, done, 0) != cudaSuccess)
     return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

@@ -17,6 +17,9 @@
 namespace attn_host {
 
 constexpr int kMaxDevices = 64;
+// attn_fwd_host overlaps its copies with the forward over at most this many
+// chunks of the problem.
+constexpr int kHostChunks = 16;
 
 struct DeviceState {
   bool ready = false;
@@ -27,6 +30,11 @@ struct DeviceState {
   uint32_t dec_attr_set = 0;       // one bit per decode kernel instantiation
   uint32_t dec_small_attr_set = 0; // one bit per small-group decode kernel instantiation
   uint32_t bwd_attr_set = 0;       // one bit per backward kernel instantiation
+  // attn_fwd_host: two copy streams and the events that order its chunks,
+  // created on its first call on the device and kept (guarded by g_host_mu)
+  bool host_ready = false;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t ev[2 * kHostChunks + 2] = {};
 };
 
 // Guards DeviceState initialisation and the per-kernel attribute bits.
@@ -35,6 +43,7 @@ extern std::atomic<unsigned long long> g_watchdog_ns;
 extern std::atomic<unsigned long long> g_launches;
 extern std::atomic<int> g_withhold;     // launches left that withhold their loads (test hook)
 extern std::atomic<unsigned long long*> g_block_count;   // block-count test hook (or nullptr)
+extern std::mutex g_host_mu;            // attn_fwd_host's streams and events
 extern PFN_cuTensorMapEncodeTiled_v12000 g_encode;
 
 inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

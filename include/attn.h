@@ -103,13 +103,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 /*
  * attn_fwd_host -- the same forward for HOST-resident inputs and outputs.
  *
- * Enqueues on `stream`: host->device copies of q, k, v into the caller's
- * device staging buffers dq, dk, dv; attn_fwd(dq, dk, dv, dout, dlse, ...);
- * device->host copies of dout into o and (when both are non-NULL) dlse into
- * lse.  Host buffers should be page-locked for the copies to be
- * asynchronous.  The caller synchronises `stream` before reading o / lse.
- * Sizes, flags and errors are those of attn_fwd; every pointer must be
- * 16-byte aligned.
+ * Copies q, k, v to the caller's device staging buffers dq, dk, dv, runs
+ * attn_fwd(dq, dk, dv, dout, dlse, ...) and copies dout back into o and
+ * (when both are non-NULL) dlse into lse.  The work is cut into up to 16
+ * chunks of consecutive (batch, K/V head) groups: the host->device copies of
+ * one chunk, the forward of the previous one (on `stream`) and the
+ * device->host copies of the one before overlap, the copies running on two
+ * copy streams the library creates once per device.  Events order the
+ * chunks, and `stream` waits for the last copy: work enqueued on `stream`
+ * later sees o and lse complete, and the caller synchronises `stream` before
+ * reading them.  Host buffers should be page-locked for the copies to be
+ * asynchronous and overlap.  Results equal attn_fwd's bitwise.  Concurrent
+ * calls from several host threads enqueue one after the other.  Sizes,
+ * flags and errors are those of attn_fwd; every pointer must be 16-byte
+ * aligned.
  */
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                   void* dq, void* dk, void* dv, void* dout, float* dlse,

@@ -232,6 +232,30 @@ def test_host_entry_point_matches_device():
     assert torch.equal(oh, o.cpu()) and torch.equal(lh, l.cpu())
 
 
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,window,n_sink", [
+    (3, 8, 2, 520, 128, 1, 0, 0),     # GQA: 6 groups, 6 chunks
+    (1, 4, 1, 333, 64, 1, 100, 5),    # MQA, G * N % 4 != 0: one chunk
+    (2, 3, 3, 257, 32, 0, 0, 0),      # 6 groups of one head, ragged N
+    (5, 8, 8, 300, 128, 1, 0, 0),     # 40 groups in 16 chunks of 2-3 groups
+])
+def test_host_entry_point_chunked_matches_device(B, H, H_kv, N, d, causal, window, n_sink):
+    """attn_fwd_host cuts the problem into chunks of (batch, K/V head) groups
+    whose copies overlap the forward: the result equals attn_fwd's bitwise."""
+    q, k, v = random_qkv(B, H, H_kv, N, d, BF, seed=21)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lh = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+    staging = {"q": torch.empty_like(q, device="cuda"), "k": torch.empty_like(k, device="cuda"),
+               "v": torch.empty_like(v, device="cuda"), "o": torch.empty_like(q, device="cuda"),
+               "lse": torch.empty(q.shape[:3], device="cuda")}
+    A.attention_from_host(qh, kh, vh, staging=staging, out=oh, lse=lh, causal=bool(causal),
+                          window=window, n_sink=n_sink)
+    torch.cuda.synchronize()
+    o, l = run_gpu(q, k, v, bool(causal), window, n_sink, A.default_scale(d), out_f32=False)
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, l.cpu())
+    assert A.get_status() == A.ATTN_OK
+
+
 def test_side_stream_and_launch_count():
     q, k, v = (t.cuda() for t in random_qkv(1, 2, 2, 333, 64, BF, seed=2))
     ref, lref = A.attention(q, k, v, causal=True)
