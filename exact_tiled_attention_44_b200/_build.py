@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 UNITS = ["attn_api.cu", "fwd_api.cu", "fwd_d128.cu", "bwd_api.cu", "decode_api.cu"]
 HEADERS = [os.path.join(CSRC, f) for f in ("host.h", "fwd_launch.cuh", "attn_kernel.cuh", "ptx.cuh", "bwd_kernel.cuh",
-                                           "decode_kernel.cuh")] + [os.path.join(ROOT, "include", "attn.h")]
+                                           "decode_tc_kernel.cuh")] + [os.path.join(ROOT, "include", "attn.h")]
 DEPS = [os.path.join(CSRC, u) for u in UNITS] + HEADERS
 OUT = os.path.join(PKG, "libattn.so")
 OBJ_DIR = os.path.join(PKG, "_objs")

@@ -1,7 +1,7 @@
 // decode_api.cu -- the split-KV decoding step: attn_decode, its workspace
 // query and attn_decode_noalloc.
 #include "host.h"
-#include "decode_kernel.cuh"
+#include "decode_tc_kernel.cuh"
 
 namespace attn_host {
 
@@ -9,34 +9,25 @@ namespace {
 
 // ------------------------------------------------------------ decode
 
-// Split rule (device independent, so that the workspace size can be queried
-// without a device): at most two CTAs per SM of a 148-SM part in total (one
-// wave; rounding the split count up would leave a short second wave), each
-// split at least 256 keys long and a whole number of 64-key tiles.
+// Workspace of attn_decode (device independent, so that its size can be
+// queried without a device, and independent of the mask): the kernel cuts
+// the kept 128-key tiles of all (batch, K/V head) groups into at most
+// DT_GRID equal ranges, so a group spans at most ceil(DT_GRID / groups) + 1
+// of them, each writing one partial result per query row.
 struct DecodePlan {
-  int n_splits, split_keys;
-  size_t counters_off, lse_off, o_off, bytes;
+  int max_parts;
+  size_t lse_off, o_off, bytes;
 };
 
 DecodePlan decode_plan(int B, int H, int H_kv, int N_q, int N_kv, int d) {
+  (void)N_kv;
   DecodePlan pl{};
   const long long groups = static_cast<long long>(B) * H_kv;
-  const long long want = groups < 296 ? 296 / groups : 1;
-  const long long max_splits = (static_cast<long long>(N_kv) + 255) / 256;
-  long long s = want < max_splits ? want : max_splits;
-  if (s < 1) s = 1;
-  const long long per = (N_kv + s - 1) / s;
-  pl.split_keys = static_cast<int>((per + attn::DEC_T - 1) / attn::DEC_T * attn::DEC_T);
-  pl.n_splits = static_cast<int>((N_kv + pl.split_keys - 1) / pl.split_keys);
-  if (pl.n_splits <= 1) {
-    pl.n_splits = 1;
-    pl.bytes = 0;
-    return pl;
-  }
-  const size_t rows = static_cast<size_t>(pl.n_splits) * B * H * N_q;
-  pl.counters_off = 0;
-  pl.lse_off = round_up(static_cast<size_t>(groups) * sizeof(int), 256);
-  pl.o_off = round_up(pl.lse_off + rows * sizeof(float), 256);
+  const long long R = static_cast<long long>(H / H_kv) * N_q;
+  pl.max_parts = static_cast<int>((attn::DT_GRID + groups - 1) / groups + 1);
+  const size_t rows = static_cast<size_t>(groups) * pl.max_parts * R;
+  pl.lse_off = 0;
+  pl.o_off = round_up(rows * sizeof(float), 256);
   pl.bytes = pl.o_off + rows * d * sizeof(float);
   return pl;
 }
@@ -60,7 +51,7 @@ int validate_decode(const void* q, const void* k, const void* v, const void* o, 
   if (H % H_kv != 0) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
-  if (static_cast<long long>(H / H_kv) * N_q > attn::DEC_MAX_ROWS) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(H / H_kv) * N_q > attn::DT_MAX_ROWS) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H_kv > 65535) return ATTN_ERR_UNSUPPORTED;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
@@ -75,70 +66,31 @@ int validate_decode(const void* q, const void* k, const void* v, const void* o, 
   return ATTN_OK;
 }
 
-// 3-D view [B*H_kv][N_kv][d] of the cache with 64 x 64 boxes, 128-byte swizzle.
-int encode_cache_map(CUtensorMap* map, const void* base, bool bf16, int d, int n, int z) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
-                              static_cast<cuuint64_t>(z)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(n) * d * 2};
-  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(attn::DEC_T), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                              3, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-template <int D, bool BF16, bool F32, int RW>
-int launch_decode_rw(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
-                     const CUtensorMap& mv, cudaStream_t stream) {
-  auto kern = attn::attn_decode_kernel<D, BF16, F32, RW>;
-  const int smem = attn::DecGeo<D>::SMEM_BYTES + 1024;
-  const int bit = (RW == 1 ? 0 : RW == 4 ? 8 : 16) + (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
+template <int D, bool BF16, bool F32>
+int launch_decode(DeviceState* st, const attn::DecTcParams& dp, const CUtensorMap& mk,
+                  const CUtensorMap& mv, bool merge, cudaStream_t stream) {
+  auto kern = attn::attn_decode_tc_kernel<D, BF16, F32>;
+  const int smem = attn::DtGeo<D>::SMEM_BYTES + 1024;
+  const int bit = (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!(st->dec_attr_set & (1u << bit))) {
+      // the kernel re-splits its registers after launch (as the forward does)
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (fa.numRegs < attn::LAUNCH_REGS) return ATTN_ERR_UNSUPPORTED;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
       st->dec_attr_set |= 1u << bit;
     }
   }
-  const dim3 grid(dp.n_splits, dp.B * dp.H_kv);
-  kern<<<grid, attn::DEC_THREADS, smem, stream>>>(mk, mv, dp);
+  kern<<<dp.grid, attn::NUM_THREADS, smem, stream>>>(mk, mv, dp);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (!merge) return ATTN_OK;
+  attn::attn_decode_tc_merge<D, BF16, F32><<<dp.n_groups, 256, 0, stream>>>(dp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-template <int D, bool BF16, bool F32, int RMAX, int NW>
-int launch_decode_small(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
-                        const CUtensorMap& mv, cudaStream_t stream) {
-  auto kern = attn::attn_decode_small_kernel<D, BF16, F32, RMAX, NW>;
-  const int smem = attn::DecSmallGeo<D, RMAX, NW>::SMEM_BYTES + 1024;
-  const int bit = (RMAX == 4 ? 0 : 8) + (D == 128 ? 4 : 0) + (BF16 ? 2 : 0) + (F32 ? 1 : 0);
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!(st->dec_small_attr_set & (1u << bit))) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-      st->dec_small_attr_set |= 1u << bit;
-    }
-  }
-  const dim3 grid(dp.n_splits, dp.B * dp.H_kv);
-  kern<<<grid, NW * 32, smem, stream>>>(mk, mv, dp);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-// Kernel by the group's query rows G * N_q: up to 4 and up to 16 rows use the
-// warp-sliced kernel, larger groups (up to 64) the row-per-warp kernel.
-template <int D, bool BF16, bool F32>
-int launch_decode(DeviceState* st, const attn::DecodeParams& dp, const CUtensorMap& mk,
-                  const CUtensorMap& mv, cudaStream_t stream) {
-  const int rows = (dp.H / dp.H_kv) * dp.N_q;
-  if (rows <= 4) return launch_decode_small<D, BF16, F32, 4, 8>(st, dp, mk, mv, stream);
-  if (rows <= 16) return launch_decode_small<D, BF16, F32, 16, 4>(st, dp, mk, mv, stream);
-  return launch_decode_rw<D, BF16, F32, 16>(st, dp, mk, mv, stream);
 }
 
 // Static decode scratch for attn_decode_noalloc: part of the module image on
@@ -173,7 +125,41 @@ int decode_impl(const void* q, const void* k, const void* v, void* o, float* lse
                            scale, dtype, &empty);
   if (rc != ATTN_OK || empty) return rc;
   const DecodePlan pl = decode_plan(B, H, H_kv, N_q, N_kv, d);
-  if (pl.n_splits > 1) {
+  attn::DecTcParams dp{};
+  dp.B = B;
+  dp.H = H;
+  dp.H_kv = H_kv;
+  dp.N_q = N_q;
+  dp.N_kv = N_kv;
+  dp.causal = causal;
+  dp.window = (window >= N_kv) ? 0 : window;
+  dp.n_sink = dp.window > 0 ? (n_sink < N_kv ? n_sink : N_kv) : 0;
+  dp.scale_log2 = scale * 1.4426950408889634f;
+  dp.R = (H / H_kv) * N_q;
+  dp.n_groups = B * H_kv;
+  // kept 128-key tiles of every group: the sink tiles, then the tiles from the
+  // first query row's window start to the end of the cache
+  dp.nt = (N_kv + attn::DT_TILE - 1) / attn::DT_TILE;
+  if (dp.window > 0) {
+    const int first = N_kv - N_q - dp.window + 1;
+    dp.wlo = first > 0 ? first / attn::DT_TILE : 0;
+    const int sb = (dp.n_sink + attn::DT_TILE - 1) / attn::DT_TILE;
+    dp.sb = sb < dp.nt ? sb : dp.nt;
+  } else {
+    dp.wlo = 0;
+    dp.sb = 0;
+  }
+  const int w0 = dp.wlo > dp.sb ? dp.wlo : dp.sb;
+  dp.tiles = dp.sb + (dp.nt > w0 ? dp.nt - w0 : 0);
+  const long long F = static_cast<long long>(dp.n_groups) * dp.tiles;
+  dp.grid = static_cast<int>(F < attn::DT_GRID ? F : attn::DT_GRID);
+  dp.max_parts = pl.max_parts;
+  // does any group span more than one range?
+  bool merge = false;
+  for (int g = 0; g < dp.n_groups && !merge; ++g)
+    merge = attn::dt_cta_of(static_cast<long long>(g) * dp.tiles, F, dp.grid) !=
+            attn::dt_cta_of(static_cast<long long>(g + 1) * dp.tiles - 1, F, dp.grid);
+  if (merge) {
     if (ws == nullptr || ws_bytes < pl.bytes) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ATTN_ERR_MISALIGNED;
     const size_t o_bytes = static_cast<size_t>(B) * H * N_q * d * ((dtype & ATTN_OUT_F32) ? 4 : 2);
@@ -190,42 +176,29 @@ int decode_impl(const void* q, const void* k, const void* v, void* o, float* lse
   const bool bf16 = (dtype & 0xF) == ATTN_BF16;
   const bool f32 = (dtype & ATTN_OUT_F32) != 0;
   alignas(64) CUtensorMap mk, mv;
-  if (encode_cache_map(&mk, k, bf16, d, N_kv, B * H_kv) != ATTN_OK ||
-      encode_cache_map(&mv, v, bf16, d, N_kv, B * H_kv) != ATTN_OK)
+  if (encode_map(&mk, k, bf16, d, N_kv, B * H_kv) != ATTN_OK ||
+      encode_map(&mv, v, bf16, d, N_kv, B * H_kv) != ATTN_OK)
     return ATTN_ERR_CUDA;
-  attn::DecodeParams dp{};
   dp.q = q;
   dp.o = o;
   dp.lse = lse;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  dp.counters = pl.n_splits > 1 ? reinterpret_cast<int*>(w + pl.counters_off) : nullptr;
-  dp.ws_lse = pl.n_splits > 1 ? reinterpret_cast<float*>(w + pl.lse_off) : nullptr;
-  dp.ws_o = pl.n_splits > 1 ? reinterpret_cast<float*>(w + pl.o_off) : nullptr;
+  dp.ws_lse = merge ? reinterpret_cast<float*>(w + pl.lse_off) : nullptr;
+  dp.ws_o = merge ? reinterpret_cast<float*>(w + pl.o_off) : nullptr;
   dp.status = st->status;
   dp.watchdog_ns = g_watchdog_ns.load(std::memory_order_relaxed);
-  dp.B = B;
-  dp.H = H;
-  dp.H_kv = H_kv;
-  dp.N_q = N_q;
-  dp.N_kv = N_kv;
-  dp.causal = causal;
-  dp.window = (window >= N_kv) ? 0 : window;
-  dp.n_sink = dp.window > 0 ? (n_sink < N_kv ? n_sink : N_kv) : 0;
-  dp.scale_log2 = scale * 1.4426950408889634f;
-  dp.n_splits = pl.n_splits;
-  dp.split_keys = pl.split_keys;
   dp.withhold_loads = take_withhold();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the per-group split counters start at zero on every call
-  if (pl.n_splits > 1 &&
-      cudaMemsetAsync(dp.counters, 0, static_cast<size_t>(B) * H_kv * sizeof(int), s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
   if (d == 128) {
-    if (bf16) return f32 ? launch_decode<128, true, true>(st, dp, mk, mv, s) : launch_decode<128, true, false>(st, dp, mk, mv, s);
-    return f32 ? launch_decode<128, false, true>(st, dp, mk, mv, s) : launch_decode<128, false, false>(st, dp, mk, mv, s);
+    if (bf16) return f32 ? launch_decode<128, true, true>(st, dp, mk, mv, merge, s)
+                         : launch_decode<128, true, false>(st, dp, mk, mv, merge, s);
+    return f32 ? launch_decode<128, false, true>(st, dp, mk, mv, merge, s)
+               : launch_decode<128, false, false>(st, dp, mk, mv, merge, s);
   }
-  if (bf16) return f32 ? launch_decode<64, true, true>(st, dp, mk, mv, s) : launch_decode<64, true, false>(st, dp, mk, mv, s);
-  return f32 ? launch_decode<64, false, true>(st, dp, mk, mv, s) : launch_decode<64, false, false>(st, dp, mk, mv, s);
+  if (bf16) return f32 ? launch_decode<64, true, true>(st, dp, mk, mv, merge, s)
+                       : launch_decode<64, true, false>(st, dp, mk, mv, merge, s);
+  return f32 ? launch_decode<64, false, true>(st, dp, mk, mv, merge, s)
+             : launch_decode<64, false, false>(st, dp, mk, mv, merge, s);
 }
 
 

@@ -166,34 +166,40 @@ int attn_alibi_slopes(int H, float* slopes);
  *   lse    device, [B, H, N_q] float32, or NULL
  *   workspace, workspace_bytes   device scratch of at least
  *          attn_decode_workspace_bytes(...) bytes, 256-byte aligned, owned by
- *          the caller and not read by it; may be NULL when that size is 0.
- *          Its counters are cleared by the call (one cudaMemsetAsync on
- *          `stream`) and it must not be shared by calls in flight at once.
+ *          the caller and not read by it; it needs no initial contents and
+ *          must not be shared by calls in flight at once.  It may be NULL
+ *          when no (batch, K/V head) group is split (see below).
  *   1 <= N_q <= N_kv; d is 64 or 128; (H / H_kv) * N_q <= 64 query rows per
  *          K/V head (else ATTN_ERR_UNSUPPORTED)
  * The mask rule, scale, dtype, LSE and error conventions are those of
- * attn_fwd, with the query position N_kv - N_q + i in place of i.  The cache
- * range is cut into splits of whole 64-key tiles; each split's partial
- * (O_s, LSE_s) goes to the workspace and the last split of each (b, kv head)
- * to finish merges them in split order (LSE = ln sum exp(LSE_s),
- * O = sum exp(LSE_s - LSE) O_s), so results are deterministic.
+ * attn_fwd, with the query position N_kv - N_q + i in place of i.  The
+ * query rows of one (batch, K/V head) group go through the tensor cores
+ * together against each 128-key tile of the cache, which is read once.  The
+ * tiles of all groups that hold a kept key are laid end to end and cut into
+ * at most 148 equal ranges, one CTA each; a group that spans several ranges
+ * gets one partial (O_s, LSE_s) per range in the workspace, and a second
+ * kernel merges them in range order (LSE = ln sum exp(LSE_s),
+ * O = sum exp(LSE_s - LSE) O_s), so results are deterministic.  One or two
+ * kernel launches on `stream`.
  */
 int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                 void* workspace, long long workspace_bytes, int B, int H, int H_kv, int N_q,
                 int N_kv, int d, int causal, int window, int n_sink, float scale, int dtype,
                 void* stream);
 
-/* Host only: bytes of workspace attn_decode needs for these sizes (0 when the
- * cache is not split), or -1 for invalid sizes.  Independent of the device. */
+/* Host only: bytes of workspace attn_decode may need for these sizes (an
+ * upper bound that depends neither on the device, the cache length nor the
+ * mask), 0 for an empty problem, or -1 for invalid sizes. */
 long long attn_decode_workspace_bytes(int B, int H, int H_kv, int N_q, int N_kv, int d);
 
 /*
  * attn_decode_noalloc -- attn_decode without a caller workspace (the paper has
- * no counterpart).  The partial results and split counters live in a static
- * 4 MiB device array that is part of the library image on every device, so
- * the call allocates nothing; its split counters are cleared on every call
- * (one cudaMemsetAsync on `stream`).  Sizes whose attn_decode_workspace_bytes
- * exceed 4 MiB return ATTN_ERR_UNSUPPORTED before anything is enqueued.
+ * no counterpart).  The partial results live in a static 4 MiB device array
+ * that is part of the library image on every device, so the call allocates
+ * nothing; nothing in the array needs to start at zero (every partial a call
+ * reads was written earlier in the same call).  Sizes whose
+ * attn_decode_workspace_bytes exceed 4 MiB return ATTN_ERR_UNSUPPORTED
+ * before anything is enqueued.
  * Races: every call on a device shares that one array, so calls on one device
  * must not overlap in time (issue them on one stream, or synchronise the
  * streams in between); overlapping calls give unspecified results.  All other

@@ -40,7 +40,10 @@ int main(void) {
   /* workspace queries */
   check("bwd_workspace_f32", attn_bwd_workspace_bytes(1, 1, 64, 64, ATTN_BF16 | ATTN_OUT_F32), 256);
   check("bwd_workspace_16", attn_bwd_workspace_bytes(1, 1, 64, 64, ATTN_BF16), 256 + 64 * 64 * 4);
-  check("decode_workspace_unsplit", attn_decode_workspace_bytes(4, 8, 2, 1, 200, 128), 0);
+  /* 8 groups: at most ceil(148 / 8) + 1 = 20 parts of 4 rows, each an LSE
+     (2560 bytes in all, already 256-aligned) and a 128-wide fp32 row */
+  check("decode_workspace", attn_decode_workspace_bytes(4, 8, 2, 1, 200, 128),
+        2560 + 20 * 8 * 4 * 128 * 4);
 
   /* invalid calls are rejected before any CUDA call */
   check("fwd_null", attn_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 64, 64, 1, 0, 0, 0.125f,

@@ -233,11 +233,18 @@ def test_decode_empty_problem_is_a_no_op():
 
 
 def test_decode_workspace_size():
-    # one split (short cache): no workspace
-    assert A.decode_workspace_bytes(4, 8, 2, 1, 200, 128) == 0
-    # split cache: counters, partial LSE and partial O for every split and row
-    b = A.decode_workspace_bytes(1, 8, 2, 1, 4096, 128)
-    assert b >= 8 * 1 * (128 + 1) * 4 * 2
+    # The kept tiles of all (batch, K/V head) groups are cut into at most 148
+    # ranges, so a group spans at most ceil(148 / groups) + 1 of them; each
+    # part keeps an LSE and a D-wide fp32 row per query row of the group.
+    for B, H, H_kv, N_q, N_kv, d in ((4, 8, 2, 1, 200, 128), (1, 8, 2, 1, 4096, 128),
+                                     (8, 32, 8, 1, 8192, 128), (1, 64, 1, 1, 20000, 64),
+                                     (300, 4, 1, 2, 100, 64)):
+        groups, rows = B * H_kv, (H // H_kv) * N_q
+        parts = -(-148 // groups) + 1
+        lse = -(-groups * parts * rows * 4 // 256) * 256
+        assert A.decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d) == lse + groups * parts * rows * d * 4
+    # it does not depend on the cache length
+    assert A.decode_workspace_bytes(1, 8, 2, 1, 4096, 128) == A.decode_workspace_bytes(1, 8, 2, 1, 64, 128)
     assert A.decode_workspace_bytes(1, 8, 2, 5, 4, 128) == -1
     assert A.decode_workspace_bytes(0, 8, 2, 1, 4096, 128) == 0
 

@@ -94,8 +94,8 @@ def test_backward_expiry_reports_timeout_and_next_call_is_correct():
 
 @pytest.mark.parametrize("H,H_kv,N_q,N_kv", [(8, 2, 1, 3000), (32, 1, 2, 1500)])
 def test_decode_expiry_reports_timeout_and_next_call_is_correct(H, H_kv, N_q, N_kv):
-    # (8, 2, 1, 3000): the small-group kernel on a split cache; (32, 1, 2, 1500):
-    # the row-per-warp kernel for a 64-row group
+    # (8, 2, 1, 3000): 4 query rows per group; (32, 1, 2, 1500): 64 rows, the
+    # largest group
     q, k, v = make_decode_inputs(1, H, H_kv, N_q, N_kv, 128, seed=6)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
     _withheld(lambda: A.decode(qd, kd, vd, causal=True))
