@@ -155,8 +155,13 @@ struct Unit {
   int n_active;
   int sb, wlo, n_iter;
   int sb0, lo0, hi0, sb1, lo1, hi1;   // per Q tile: sink prefix, window range
+  int last0, last1;                   // per Q tile: the last block it visits
 };
 
+// REV: blocks are visited in descending order.  The forward does so under a
+// position bias: the bias grows towards the diagonal, so the nearest keys come
+// first and the running row max seldom has to move (each move rescales O).
+template <bool REV>
 __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
   Unit U;
   const int BH = p.B * p.H;
@@ -196,6 +201,12 @@ __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
   U.sb = sb;
   U.wlo = max(lo_min, sb);
   U.n_iter = sb + max(0, hi_max - U.wlo);
+  // Visited blocks: [0, sb) then [wlo, hi_max).  In ascending order a tile's
+  // last block is hi - 1; in descending order it is its lowest visited block:
+  // 0 with sink blocks, else lo (visited as a sink-prefix block when lo < sb,
+  // otherwise from wlo on).
+  U.last0 = REV ? (U.sb0 > 0 ? 0 : (U.lo0 < sb ? U.lo0 : max(U.lo0, U.wlo))) : U.hi0 - 1;
+  U.last1 = REV ? (U.sb1 > 0 ? 0 : (U.lo1 < sb ? U.lo1 : max(U.lo1, U.wlo))) : U.hi1 - 1;
   return U;
 }
 
@@ -216,8 +227,10 @@ __device__ __forceinline__ int num_rounds(int grid, int num_units) {
 // Q slot of tile t in the CTA's ul-th unit.
 __device__ __forceinline__ int q_slot(int ul, int t) { return (2 * ul + t) % Q_SLOTS; }
 
+template <bool REV>
 __device__ __forceinline__ int block_at(const Unit& U, int idx) {
-  return idx < U.sb ? idx : U.wlo + (idx - U.sb);
+  const int k = REV ? U.n_iter - 1 - idx : idx;
+  return k < U.sb ? k : U.wlo + (k - U.sb);
 }
 
 __device__ __forceinline__ bool tile_uses(const Unit& U, int t, int j) {
@@ -228,7 +241,7 @@ __device__ __forceinline__ bool tile_uses(const Unit& U, int t, int j) {
 }
 
 __device__ __forceinline__ int tile_last_block(const Unit& U, int t) {
-  return (t == 0 ? U.hi0 : U.hi1) - 1;
+  return t == 0 ? U.last0 : U.last1;
 }
 
 // True when some (row, key) of Q tile rows [r0, r0+128) x keys [c0, c0+128)
@@ -330,7 +343,7 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)
 
 // ------------------------------------------------------------ roles
 
-template <int D>
+template <int D, bool REV>
 __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                          const CUtensorMap* tmV, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
@@ -366,7 +379,7 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit(u, p);
+    const Unit U = decode_unit<REV>(u, p);
     // Loads in the order their ring stages and Q slots are released, so
     // that no load waits behind one whose slot frees later: Q tile 0 (its
     // slot was released by the unit before last), the first K block (whose
@@ -377,7 +390,7 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
     if (!ok) break;
     const int kvz = U.b * p.H_kv + U.g;
     for (int idx = 0; idx < U.n_iter; ++idx, ++kv_it) {
-      const int j = block_at(U, idx);
+      const int j = block_at<REV>(U, idx);
       const int s = kv_it % NUM_STAGES;
       const uint32_t ph = (kv_it / NUM_STAGES) & 1u;
       ok = warp_wait(bars + 8 * (B_K_EMPTY + s), ph ^ 1u, abort_flag, p);
@@ -455,7 +468,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int t, i
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool REV>
 __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
   uint32_t kv_it = 0, p_ph[2] = {0, 0};
@@ -470,7 +483,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit(u, p);
+    const Unit U = decode_unit<REV>(u, p);
     const int qs0 = q_slot(ul, 0), qs1 = q_slot(ul, 1);
     auto wait_q = [&](int qs) {
       if (!warp_wait(bars + 8 * (B_Q_FULL + qs), q_uses[qs] & 1u, abort_flag, p)) return false;
@@ -494,7 +507,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       u_next = unit_of_round(r2, blockIdx.x, gridDim.x, p.num_units);
     // prologue: S_t for the first block
     {
-      const int j0 = block_at(U, 0);
+      const int j0 = block_at<REV>(U, 0);
       const int s = kv_it % NUM_STAGES;
       ok = warp_wait(bars + 8 * (B_K_FULL + s), (kv_it / NUM_STAGES) & 1u, abort_flag, p);
       if (!ok) break;
@@ -523,13 +536,13 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
     }
     int pv_done[2] = {0, 0};
     for (int idx = 0; idx < U.n_iter && ok; ++idx) {
-      const int j = block_at(U, idx);
+      const int j = block_at<REV>(U, idx);
       const uint32_t it = kv_it + idx;
       const int s = it % NUM_STAGES;
       ok = warp_wait(bars + 8 * (B_V_FULL + s), (it / NUM_STAGES) & 1u, abort_flag, p);
       if (!ok) break;
       const bool has_next = idx + 1 < U.n_iter;
-      const int jn = has_next ? block_at(U, idx + 1) : 0;
+      const int jn = has_next ? block_at<REV>(U, idx + 1) : 0;
       const uint32_t itn = it + 1;
       const int sn = itn % NUM_STAGES;
       // Q tile 0: P0 V_j, then S0 for the next block
@@ -599,10 +612,9 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       // issue it now, so that softmax 0 finds it ready after its epilogue
       // instead of waiting for tile 1 to finish this unit.  S_0 overwrites
       // P_0 only after the P_0 V issued before it (the pipe runs in order).
-      if (!s0_pre && u_next >= 0 && has_next && j >= tile_last_block(U, 0) &&
-          idx + 2 == U.n_iter) {
-        const Unit UN = decode_unit(u_next, p);
-        const int jn0 = block_at(UN, 0);
+      if (!s0_pre && u_next >= 0 && has_next && !tile_uses(U, 0, jn) && idx + 2 == U.n_iter) {
+        const Unit UN = decode_unit<REV>(u_next, p);
+        const int jn0 = block_at<REV>(UN, 0);
         if (tile_uses(UN, 0, jn0)) {
           const uint32_t it2 = kv_it + U.n_iter;       // ring position of the next unit's first K
           const int s2 = it2 % NUM_STAGES;
@@ -666,7 +678,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     ++ul;
-    const Unit U = decode_unit(u, p);
+    const Unit U = decode_unit<ALIBI>(u, p);
     if (t >= U.n_active) continue;
     const int r0 = U.q0 + t * BM;
     const int row = r0 + row_in_tile;
@@ -676,7 +688,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     float m_run = -INFINITY, l_exact = 0.f, l_round = 0.f;
     bool first = true;
     for (int idx = 0; idx < U.n_iter; ++idx) {
-      const int j = block_at(U, idx);
+      const int j = block_at<ALIBI>(U, idx);
       if (!tile_uses(U, t, j)) continue;
       release_stage();
       // one verdict for the whole warp: the TMEM load and the vote below are
@@ -690,8 +702,24 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       const int c0 = j * BN;
       const bool masked = block_needs_mask(p, r0, c0);
       float m_blk;
+      // ALiBi on a block whose kept keys all lie on one side of every row of
+      // the tile: the bias -slope |i - j| is linear in the block-local
+      // key index e, so it folds into the raw scores as y = s + sigma e'
+      // (sigma = slope / scale, e' = e for keys at or before the rows,
+      // BN - 1 - e for keys at or after them), and the logit is c y + kappa
+      // with one constant kappa per row.
+      bool linear = false, after = false;
+      float kappa = 0.f;
+      if constexpr (ALIBI) {
+        // under the causal mask every kept key is at or before its row
+        const bool before = p.causal || c0 + BN - 1 <= r0;
+        after = !before && c0 >= r0 + BM - 1;
+        linear = (before || after) && c != 0.f && fabsf(slope2 / c) < 1e30f;
+        const float relf = static_cast<float>(row - c0);   // exact in fp32
+        if (linear) kappa = after ? slope2 * (relf - static_cast<float>(BN - 1)) : -slope2 * relf;
+      }
       // Logits already scaled (and biased) in sr, instead of raw scores.
-      const bool prescaled = ALIBI || (masked && c == 0.f);
+      const bool prescaled = (ALIBI && !linear) || (masked && c == 0.f);
       if (prescaled) {
         // Scale first (adding the position bias -slope |i - j|), then drop
         // masked keys with -inf (any sign of scale).  Kept keys of this row,
@@ -701,32 +729,15 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
         const int lo = p.window > 0 ? row - p.window + 1 - c0 : -(1 << 30);
         const int sk = p.window > 0 ? p.n_sink - c0 : -(1 << 30);
         const float rel = static_cast<float>(row - c0);   // i - c0, exact in fp32
-        if (ALIBI && !masked && p.causal) {
-          // Every key of an unmasked causal block is at or before the row, so
-          // |i - j| = rel - e >= 0: the distance is formed exactly (small
-          // integers), then scaled by the slope once.
-          const float2 rel2 = make_float2(rel, rel);
-          const float2 nsl2 = make_float2(-slope2, -slope2);
-          const float2 c2 = make_float2(c, c);
 #pragma unroll
-          for (int e = 0; e < 128; e += 2) {
-            const float2 dist = sub2(rel2, make_float2(static_cast<float>(e), static_cast<float>(e + 1)));
-            const float2 s2 = make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
-            const float2 x = fma2(dist, nsl2, mul2(s2, c2));
-            sr[e] = __float_as_uint(x.x);
-            sr[e + 1] = __float_as_uint(x.y);
+        for (int e = 0; e < 128; ++e) {
+          float x = __uint_as_float(sr[e]) * c;
+          if constexpr (ALIBI) x = fmaf(-slope2, fabsf(rel - static_cast<float>(e)), x);
+          if (masked) {
+            const bool keep = (e <= hi) && (e >= lo || e < sk);
+            x = keep ? x : -INFINITY;
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            float x = __uint_as_float(sr[e]) * c;
-            if constexpr (ALIBI) x = fmaf(-slope2, fabsf(rel - static_cast<float>(e)), x);
-            if (masked) {
-              const bool keep = (e <= hi) && (e >= lo || e < sk);
-              x = keep ? x : -INFINITY;
-            }
-            sr[e] = __float_as_uint(x);
-          }
+          sr[e] = __float_as_uint(x);
         }
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
@@ -766,8 +777,20 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
             for (int e = 0; e < 128; ++e) sr[e] = ((e <= hi) && (e >= lo || e < sk)) ? sr[e] : gone;
           }
         }
+        if (ALIBI && linear) {
+          const float sigma = slope2 / c;
+          if (after) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              sr[e] = __float_as_uint(fmaf(sigma, static_cast<float>(BN - 1 - e), __uint_as_float(sr[e])));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              sr[e] = __float_as_uint(fmaf(sigma, static_cast<float>(e), __uint_as_float(sr[e])));
+          }
+        }
         // raw-score extreme, then one multiply: max of s*c is c*max(s) for c >= 0
-        // and c*min(s) for c < 0
+        // and c*min(s) for c < 0 (plus the row constant of a linear ALiBi block)
         float m0 = __uint_as_float(sr[0]), m1 = __uint_as_float(sr[1]);
         if (c >= 0.f) {
 #pragma unroll
@@ -776,7 +799,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
             m1 = max3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
           }
           m0 = max3(m0, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
-          m_blk = fmaxf(m0, m1) * c;
+          m_blk = fmaf(fmaxf(m0, m1), c, kappa);
         } else {
 #pragma unroll
           for (int e = 2; e < 126; e += 4) {
@@ -784,7 +807,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
             m1 = min3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
           }
           m0 = min3(m0, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
-          m_blk = fminf(m0, m1) * c;
+          m_blk = fmaf(fminf(m0, m1), c, kappa);
         }
       }
       // online softmax update (log2 units); lazy rescale
@@ -797,7 +820,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
       const float2 cc2 = prescaled ? make_float2(1.f, 1.f) : make_float2(c, c);
-      const float2 nm2 = make_float2(-mref, -mref);
+      const float2 nm2 = make_float2(kappa - mref, kappa - mref);
       // Two denominators: le sums the fp32 weights (for the LSE), lr sums the
       // same 16-bit-rounded weights the P V MMA consumes (for O, so that every
       // output row is a convex combination of V rows under those weights).
@@ -994,6 +1017,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     tma_prefetch_desc(&tmV);
     if (!OUT_F32) tma_prefetch_desc(&tmO);
   }
+  // The set-up above touches no global memory, so it may overlap the end of
+  // the previous grid of the stream; nothing below runs before that grid is done.
+  grid_dependency_wait();
+  grid_launch_dependents();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -1011,9 +1038,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else {
     regs_decrease<CONTROL_REGS>();
     if (warp == MMA_WARP) {
-      mma_role<D, BF16>(p, tmem, sbase, bars, abort_flag);
+      mma_role<D, BF16, ALIBI>(p, tmem, sbase, bars, abort_flag);
     } else if (warp == TMA_WARP) {
-      tma_role<D>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
+      tma_role<D, ALIBI>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();

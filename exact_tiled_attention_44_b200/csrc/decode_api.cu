@@ -84,13 +84,13 @@ int launch_decode(DeviceState* st, const attn::DecTcParams& dp, const CUtensorMa
       st->dec_attr_set |= 1u << bit;
     }
   }
-  kern<<<dp.grid, attn::NUM_THREADS, smem, stream>>>(mk, mv, dp);
+  cudaError_t e = launch_overlapped(kern, dp.grid, attn::NUM_THREADS, smem, stream, mk, mv, dp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (!merge) return ATTN_OK;
-  attn::attn_decode_tc_merge<D, BF16, F32><<<dp.n_groups, 256, 0, stream>>>(dp);
+  e = launch_overlapped(attn::attn_decode_tc_merge<D, BF16, F32>, dp.n_groups, 256, 0, stream, dp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 // Static decode scratch for attn_decode_noalloc: part of the module image on

@@ -574,6 +574,10 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
+  // The set-up above touches no global memory, so it may overlap the end of
+  // the previous grid of the stream; nothing below runs before that grid is done.
+  grid_dependency_wait();
+  grid_launch_dependents();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -613,25 +617,27 @@ attn_decode_tc_merge(const DecTcParams p) {
   if (n_parts <= 1) return;
   const int b = g / p.H_kv, gk = g % p.H_kv;
   const int G_heads = p.H / p.H_kv;
+  // launched behind the split kernel, whose partials it reads (through L2)
+  grid_dependency_wait();
   for (int idx = threadIdx.x; idx < p.R * (D / 4); idx += blockDim.x) {
     const int r = idx / (D / 4), c4 = idx % (D / 4);
     const size_t row_idx = ((static_cast<size_t>(b) * p.H + gk * G_heads + r / p.N_q) * p.N_q) + r % p.N_q;
     const float* ls = p.ws_lse + static_cast<size_t>(g) * p.max_parts * p.R + r;   // stride R
     float mx = -INFINITY;
-    for (int s = 0; s < n_parts; ++s) mx = fmaxf(mx, __ldg(ls + static_cast<size_t>(s) * p.R));
+    for (int s = 0; s < n_parts; ++s) mx = fmaxf(mx, __ldcg(ls + static_cast<size_t>(s) * p.R));
     float tot = 0.f;
     for (int s = 0; s < n_parts; ++s) {
-      const float l = __ldg(ls + static_cast<size_t>(s) * p.R);
+      const float l = __ldcg(ls + static_cast<size_t>(s) * p.R);
       tot += (l == -INFINITY) ? 0.f : __expf(l - mx);
     }
     const float lse_nat = (mx == -INFINITY) ? -INFINITY : mx + __logf(tot);
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < n_parts; ++s) {
       const size_t sl = (static_cast<size_t>(g) * p.max_parts + s) * p.R + r;
-      const float l = __ldg(p.ws_lse + sl);
+      const float l = __ldcg(p.ws_lse + sl);
       if (l == -INFINITY) continue;
       const float wgt = __expf(l - lse_nat);
-      const float4 x = __ldg(reinterpret_cast<const float4*>(p.ws_o + sl * D) + c4);
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.ws_o + sl * D) + c4);
       o.x = fmaf(wgt, x.x, o.x);
       o.y = fmaf(wgt, x.y, o.y);
       o.z = fmaf(wgt, x.z, o.z);

@@ -30,9 +30,9 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
     }
   }
   const int grid = kp.num_units < st->sm_count ? kp.num_units : st->sm_count;
-  kern<<<grid, attn::NUM_THREADS, smem, stream>>>(mq, mk, mv, mo, kp);
+  const cudaError_t e = launch_overlapped(kern, grid, attn::NUM_THREADS, smem, stream, mq, mk, mv, mo, kp);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, bool ALIBI>

@@ -11,6 +11,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "attn.h"
 
@@ -75,6 +76,26 @@ int device_state(DeviceState** out);
 // 3-D view [z][rows][d] of a contiguous [.., n, d] 16-bit tensor; box =
 // (min(d, 64), 128, 1) with the swizzle span equal to the box's row bytes.
 int encode_map(CUtensorMap* map, const void* base, bool bf16, int d, int n, int z);
+
+// Launches `kern` with programmatic stream serialisation: its CTAs may be
+// scheduled while the previous grid of the stream drains, run their set-up
+// (barriers, TMEM, descriptor prefetch) and then wait for that grid in
+// grid_dependency_wait before their first memory access.
+template <typename... Params, typename... Args>
+cudaError_t launch_overlapped(void (*kern)(Params...), int grid, int block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Takes one launch from the withhold-loads test hook, if any is pending.
 int take_withhold();

@@ -71,6 +71,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// ------------------------------------------------- dependent launches
+
+// Waits until every grid this one was launched behind (with programmatic
+// stream serialisation) has completed and its memory writes are visible.
+// Without that launch attribute the stream order already holds and this
+// returns at once.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allows the next grid of the stream, if it was launched with programmatic
+// stream serialisation, to be scheduled once every CTA of this grid has
+// issued this (or exited).  That grid still waits in grid_dependency_wait for
+// this one to complete before it touches memory.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

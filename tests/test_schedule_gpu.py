@@ -48,6 +48,18 @@ def test_forward_computes_exactly_the_visited_blocks(case):
 
 
 @pytest.mark.parametrize("case", CASES)
+def test_forward_with_position_bias_computes_exactly_the_visited_blocks(case):
+    """With ALiBi slopes the forward walks every unit's blocks in descending
+    order; the set of score tiles it computes is the same."""
+    B, H, H_kv, N, d, dt, causal, window, n_sink = case
+    q, k, v = (t.cuda() for t in random_qkv(B, H, H_kv, N, d, dt, seed=1))
+    s = A.alibi_slopes(H, "cuda")
+    got = _count(lambda: A.attention(q, k, v, causal=bool(causal), window=window, n_sink=n_sink,
+                                     alibi_slopes=s))
+    assert got == A.visited_blocks(N, bool(causal), window, n_sink) * B * H
+
+
+@pytest.mark.parametrize("case", CASES)
 def test_backward_steps_are_exactly_the_visited_blocks(case):
     B, H, H_kv, N, d, dt, causal, window, n_sink = case
     q, k, v = (t.cuda() for t in random_qkv(B, H, H_kv, N, d, dt, seed=1))
