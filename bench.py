@@ -370,23 +370,24 @@ def decode_bench(args):
     sampler = ClockSampler(dev.index if dev.index is not None else 0, args.clocks_csv)
     sampler.start()
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    # Steps run back to back, as in a decoding loop: no event between them
+    # (an event between two launches would also stop the next step's set-up
+    # from overlapping the end of the previous one).  The two input sets
+    # together exceed L2, so every step reads its cache from HBM.
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     n0 = A.launch_count()
     sampler.mark_begin()
     t0.record(stream)
     for i in range(K):
-        ev[i][0].record(stream)
         step(i)
-        ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.mark_end()
     launches = A.launch_count() - n0
     clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    kern_ms = total_ms / K
     peaks = load_peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     line = {
@@ -403,7 +404,9 @@ def decode_bench(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peaks['source']} HBM copy (MEASURED_PEAKS.json)",
-                     "kernel_ms": kern_ms},
+                     "kernel_ms": kern_ms,
+                     "kernel_ms_scope": "one decoding step (split kernel and, when groups are "
+                                        "split, the merge kernel), averaged over the timed steps"},
         "gpu_launches": launches,
         "clocks": clocks,
         "device_status": A.get_status(),

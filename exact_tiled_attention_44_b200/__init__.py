@@ -25,7 +25,7 @@ __all__ = [
     "attn_decode_noalloc_raw", "attention_backward", "attn_bwd_raw", "bwd_workspace_bytes",
     "unmasked_pairs",
     "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
-    "test_count_blocks", "error_string",
+    "test_count_blocks", "test_force_units", "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
     "ATTN_BF16", "ATTN_FP16", "ATTN_OUT_F32",
@@ -45,8 +45,8 @@ EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_s
                     "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
-                    "attn_test_withhold_loads", "attn_test_count_blocks", "attn_bwd",
-                    "attn_bwd_workspace_bytes")
+                    "attn_test_withhold_loads", "attn_test_count_blocks", "attn_test_force_units",
+                    "attn_bwd", "attn_bwd_workspace_bytes")
 
 _LIB = None
 
@@ -101,6 +101,8 @@ def load_library():
     lib.attn_test_withhold_loads.restype = ci
     lib.attn_test_count_blocks.argtypes = [vp]
     lib.attn_test_count_blocks.restype = ci
+    lib.attn_test_force_units.argtypes = [ci]
+    lib.attn_test_force_units.restype = ci
     lib.attn_bwd.argtypes = [vp] * 11 + [ctypes.c_longlong] + [ci] * 8 + [cf, ci, vp]
     lib.attn_bwd.restype = ci
     lib.attn_bwd_workspace_bytes.argtypes = [ci] * 5
@@ -140,6 +142,13 @@ def test_withhold_loads(n_launches: int) -> int:
     """Failure-detection hook: the next n launches issue no copies, so their
     waits run into the watchdog (see include/attn.h)."""
     return int(load_library().attn_test_withhold_loads(int(n_launches)))
+
+
+def test_force_units(mode: int) -> int:
+    """Work-unit shape hook for tests: 0 forces pairs of Q tiles, 1 single
+    tiles shared by both softmax warpgroups, -1 the automatic choice (see
+    include/attn.h)."""
+    return int(load_library().attn_test_force_units(int(mode)))
 
 
 def test_count_blocks(counter: torch.Tensor | None) -> int:

@@ -24,6 +24,7 @@ std::mutex g_mu;
 std::atomic<unsigned long long> g_watchdog_ns{2000000000ull};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<int> g_withhold{0};
+std::atomic<int> g_force_units{-1};
 std::atomic<unsigned long long*> g_block_count{nullptr};
 std::mutex g_host_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -173,6 +174,9 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   // the last copy, so the contract of a single stream holds.
   const long long groups = static_cast<long long>(B) * H_kv;
   const int G = H / H_kv;
+  // every chunk runs the work-unit shape attn_fwd would choose for the whole problem
+  const int forced = g_force_units.load();
+  const bool split = forced >= 0 ? forced == 1 : fwd_split_units(B, H, N, false, st->sm_count);
   // chunked LSE rows must keep the 16-byte alignment attn_fwd requires
   const bool lse_ok = !with_lse || (static_cast<long long>(G) * N) % 4 == 0;
   const int n_chunks = lse_ok ? static_cast<int>(groups < kHostChunks ? groups : kHostChunks) : 1;
@@ -213,8 +217,8 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
         cudaMemcpyAsync(dvc, at(v, g0 * kv_grp), T * kv_grp, cudaMemcpyHostToDevice, st->copy_in) != cudaSuccess ||
         cudaEventRecord(in, st->copy_in) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    rc = attn_fwd(dqc, dkc, dvc, doc, dlc, static_cast<int>(T), G, 1, N, d, causal, window, n_sink,
-                  scale, dtype, stream);
+    rc = fwd_impl(dqc, dkc, dvc, doc, dlc, nullptr, static_cast<int>(T), G, 1, N, d, causal, window,
+                  n_sink, scale, dtype, stream, split ? 1 : 0);
     if (rc != ATTN_OK) return rc;
     if (cudaEventRecord(out, s) != cudaSuccess || cudaStreamWaitEvent(st->copy_out, out, 0) != cudaSuccess ||
         cudaMemcpyAsync(const_cast<char*>(at(o, g0 * o_grp)), doc, T * o_grp, cudaMemcpyDeviceToHost,
@@ -313,6 +317,12 @@ int attn_test_withhold_loads(int n_launches) {
 
 int attn_test_count_blocks(unsigned long long* counter) {
   g_block_count.store(counter);
+  return ATTN_OK;
+}
+
+int attn_test_force_units(int mode) {
+  if (mode < -1 || mode > 1) return ATTN_ERR_INVALID_ARG;
+  g_force_units.store(mode);
   return ATTN_OK;
 }
 

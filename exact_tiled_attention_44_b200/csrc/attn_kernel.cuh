@@ -71,8 +71,9 @@ struct KernelParams {
   int causal, window, n_sink;
   float scale_log2;   // scale * log2(e)
   int n_qpairs;       // ceil(N / 256)
+  int n_qtiles;       // ceil(N / 128)
   int n_kblocks;      // ceil(N / 128)
-  int num_units;      // B * H * n_qpairs
+  int num_units;      // B * H * n_qpairs (pair units) or B * H * n_qtiles (split units)
   const float* alibi; // ALiBi slope per query head ([H], device), used by the ALIBI kernels
   int withhold_loads; // test hook: the TMA warp issues nothing, so every wait runs out
   unsigned long long* block_count;  // test hook: S tiles computed are added here (or nullptr)
@@ -97,7 +98,10 @@ struct Geo {
   static constexpr int K_OFF = Q_OFF + Q_SLOTS * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + NUM_STAGES * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + NUM_STAGES * TILE_BYTES;
-  static constexpr int SMEM_BYTES = BAR_OFF + 256;
+  // split units: softmax warpgroup 1 hands (m, l_exact, l_round) of each row
+  // to warpgroup 0, which merges the two halves
+  static constexpr int STATS_OFF = BAR_OFF + 256;
+  static constexpr int SMEM_BYTES = STATS_OFF + 128 * 12;
   static constexpr uint32_t S_COL0 = 0;      // S_t at column 128 t
   static constexpr uint32_t O_COL0 = 256;    // O_t at column 256 + D t
   static_assert(D % 16 == 0 && D <= 128, "unsupported head dim");
@@ -115,7 +119,9 @@ enum BarSlot : int {
   B_O_FULL = B_P_FULL + 2,             // [2]
   B_DRAIN = B_O_FULL + 2,
   B_EPI = B_DRAIN + 1,                 // [2] a tile's output rows are staged in shared memory
-  B_COUNT = B_EPI + 2
+  B_HALF = B_EPI + 2,                  // split units: warpgroup 1's row statistics are written
+  B_HALF_FREE = B_HALF + 1,            // split units: warpgroup 0 has read them and O_1
+  B_COUNT = B_HALF_FREE + 1
 };
 constexpr int TMEM_SLOT_OFF = 8 * B_COUNT;
 constexpr int ABORT_FLAG_OFF = TMEM_SLOT_OFF + 4;
@@ -161,24 +167,31 @@ struct Unit {
 // REV: blocks are visited in descending order.  The forward does so under a
 // position bias: the bias grows towards the diagonal, so the nearest keys come
 // first and the running row max seldom has to move (each move rescales O).
-template <bool REV>
+//
+// SPLIT: a unit is one Q tile instead of a pair, and the two softmax
+// warpgroups ("tiles" t = 0, 1 below) share its rows: t takes the visited
+// blocks at even (t = 0) or odd (t = 1) positions, with its own S_t, O_t and
+// running (m, l); warpgroup 0 merges the halves in the epilogue.  Used when
+// pair units would leave SMs idle (few heads, short sequences).
+template <bool REV, bool SPLIT>
 __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
+  static_assert(!(REV && SPLIT), "split units visit blocks in ascending order");
   Unit U;
   const int BH = p.B * p.H;
-  // Longest-processing-time first: causal cost grows with the pair index, so
-  // units are handed out from the last pair of every head down to the first.
-  const int pair = p.n_qpairs - 1 - u / BH;
+  // Longest-processing-time first: causal cost grows with the pair (tile)
+  // index, so units are handed out from the last pair of every head down.
+  const int pair = (SPLIT ? p.n_qtiles : p.n_qpairs) - 1 - u / BH;
   U.bh = u % BH;
   U.b = U.bh / p.H;
   U.h = U.bh % p.H;
   U.g = U.h / (p.H / p.H_kv);
-  U.q0 = pair * 2 * BM;
-  U.n_active = (U.q0 + BM < p.N) ? 2 : 1;
+  U.q0 = pair * (SPLIT ? 1 : 2) * BM;
+  U.n_active = (!SPLIT && U.q0 + BM < p.N) ? 2 : 1;
   const int sink_blocks = (p.window > 0) ? (p.n_sink + BN - 1) / BN : 0;
   int sb = 0, lo_min = 1 << 30, hi_max = 0;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int r0 = U.q0 + t * BM;
+    const int r0 = U.q0 + (SPLIT ? 0 : t * BM);
     const int r_last = min(r0 + BM - 1, p.N - 1);
     int lo = 0, hi = p.n_kblocks;
     if (p.causal) hi = min(p.n_kblocks, r_last / BN + 1);
@@ -207,6 +220,14 @@ __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
   // otherwise from wlo on).
   U.last0 = REV ? (U.sb0 > 0 ? 0 : (U.lo0 < sb ? U.lo0 : max(U.lo0, U.wlo))) : U.hi0 - 1;
   U.last1 = REV ? (U.sb1 > 0 ? 0 : (U.lo1 < sb ? U.lo1 : max(U.lo1, U.wlo))) : U.hi1 - 1;
+  if constexpr (SPLIT) {
+    // every visited block holds kept keys of the tile's rows; the last even
+    // and the last odd position (none for t = 1 when only one block is visited)
+    const int i0 = (U.n_iter - 1) & ~1;
+    const int i1 = (U.n_iter - 1) & 1 ? U.n_iter - 1 : U.n_iter - 2;
+    U.last0 = i0 < U.sb ? i0 : U.wlo + (i0 - U.sb);
+    U.last1 = i1 < 0 ? -1 : (i1 < U.sb ? i1 : U.wlo + (i1 - U.sb));
+  }
   return U;
 }
 
@@ -233,7 +254,12 @@ __device__ __forceinline__ int block_at(const Unit& U, int idx) {
   return k < U.sb ? k : U.wlo + (k - U.sb);
 }
 
+template <bool SPLIT>
 __device__ __forceinline__ bool tile_uses(const Unit& U, int t, int j) {
+  if constexpr (SPLIT) {
+    const int idx = j < U.sb ? j : U.sb + (j - U.wlo);   // position of visited block j
+    return (idx & 1) == t;
+  }
   const int sb = t == 0 ? U.sb0 : U.sb1;
   const int lo = t == 0 ? U.lo0 : U.lo1;
   const int hi = t == 0 ? U.hi0 : U.hi1;
@@ -334,6 +360,23 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[W]) {
   else tmem_ld_32x32b_x16(taddr, r);
 }
 
+// Split units: o0 <- o0 w0 + o1 w1 over W columns, o1 read from TMEM at
+// taddr1 when the other half holds a sum (has1), else o0 <- o0 w0.
+template <int W>
+__device__ __forceinline__ void merge_half(uint32_t (&o0)[W], uint32_t taddr1, bool has1, float w0,
+                                           float w1) {
+  if (has1) {
+    uint32_t o1[W];
+    tmem_ld_cols<W>(taddr1, o1);
+#pragma unroll
+    for (int e = 0; e < W; ++e)
+      o0[e] = __float_as_uint(fmaf(__uint_as_float(o0[e]), w0, __uint_as_float(o1[e]) * w1));
+  } else {
+#pragma unroll
+    for (int e = 0; e < W; ++e) o0[e] = __float_as_uint(__uint_as_float(o0[e]) * w0);
+  }
+}
+
 template <int W>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[W]) {
   if constexpr (W == 32) tmem_st_32x32b_x32(taddr, r);
@@ -343,7 +386,7 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)
 
 // ------------------------------------------------------------ roles
 
-template <int D, bool REV>
+template <int D, bool REV, bool SPLIT>
 __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                          const CUtensorMap* tmV, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
@@ -379,7 +422,7 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit<REV>(u, p);
+    const Unit U = decode_unit<REV, SPLIT>(u, p);
     // Loads in the order their ring stages and Q slots are released, so
     // that no load waits behind one whose slot frees later: Q tile 0 (its
     // slot was released by the unit before last), the first K block (whose
@@ -468,7 +511,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int t, i
   }
 }
 
-template <int D, bool BF16, bool REV>
+template <int D, bool BF16, bool REV, bool SPLIT>
 __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
   uint32_t kv_it = 0, p_ph[2] = {0, 0};
@@ -483,8 +526,9 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit<REV>(u, p);
-    const int qs0 = q_slot(ul, 0), qs1 = q_slot(ul, 1);
+    const Unit U = decode_unit<REV, SPLIT>(u, p);
+    // split units: both tiles read the unit's one Q tile
+    const int qs0 = q_slot(ul, 0), qs1 = SPLIT ? qs0 : q_slot(ul, 1);
     auto wait_q = [&](int qs) {
       if (!warp_wait(bars + 8 * (B_Q_FULL + qs), q_uses[qs] & 1u, abort_flag, p)) return false;
       ++q_uses[qs];
@@ -496,9 +540,10 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
     const bool this_s0_pre = s0_pre;
     s0_pre = false;
     auto need_q = [&](int t) {
-      if (q_ready[t]) return true;
-      if (!wait_q(t == 0 ? qs0 : qs1)) return false;
-      q_ready[t] = true;
+      const int tq = SPLIT ? 0 : t;
+      if (q_ready[tq]) return true;
+      if (!wait_q(tq == 0 ? qs0 : qs1)) return false;
+      q_ready[tq] = true;
       return true;
     };
     // the CTA's next unit, for issuing its first S_0 early
@@ -513,7 +558,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       if (!ok) break;
       tc_fence_after_sync();
       for (int t = 0; t < 2 && ok; ++t) {
-        if (!tile_uses(U, t, j0)) continue;
+        if (!tile_uses<SPLIT>(U, t, j0)) continue;
         if (t == 0 && this_s0_pre) continue;        // issued at the end of the unit before
         ok = need_q(t);
         if (!ok) break;
@@ -535,6 +580,69 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       __syncwarp();
     }
     int pv_done[2] = {0, 0};
+    if constexpr (SPLIT) {
+      // Split unit: block idx belongs to tile t = idx & 1 and the next one to
+      // the other tile, whose S does not wait for P_t: it is issued first, so
+      // that the other warpgroup's softmax overlaps this one's.
+      for (int idx = 0; idx < U.n_iter && ok; ++idx) {
+        const int j = block_at<REV>(U, idx);
+        const int t = idx & 1;
+        const uint32_t it = kv_it + idx;
+        const int s = it % NUM_STAGES;
+        const bool has_next = idx + 1 < U.n_iter;
+        if (has_next) {
+          const uint32_t itn = it + 1;
+          const int sn = itn % NUM_STAGES;
+          ok = warp_wait(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
+          if (!ok) break;
+          tc_fence_after_sync();
+          ok = need_q(1 - t);
+          if (!ok) break;
+          if (elect_one()) {
+            // S_{1-t} overwrites P_{1-t} after the P_{1-t} V issued before it
+            issue_qk<D, BF16>(tmem, sbase, 1 - t, qs0, sn);
+            mma_commit(bars + 8 * (B_S_FULL + 1 - t));
+            mma_commit(bars + 8 * (B_K_EMPTY + sn));
+            if (idx + 2 == U.n_iter) mma_commit(bars + 8 * (B_Q_EMPTY + qs0));   // last S of the unit
+          }
+          __syncwarp();
+          ++n_s;
+        }
+        ok = warp_wait(bars + 8 * (B_V_FULL + s), (it / NUM_STAGES) & 1u, abort_flag, p);
+        if (!ok) break;
+        ok = warp_wait(bars + 8 * (B_P_FULL + t), p_ph[t], abort_flag, p);
+        if (!ok) break;
+        p_ph[t] ^= 1u;
+        tc_fence_after_sync();
+        if (elect_one()) {
+          issue_pv<D, BF16>(tmem, sbase, t, s, pv_done[t] > 0);
+          if (j == tile_last_block(U, t)) mma_commit(bars + 8 * (B_O_FULL + t));
+          mma_commit(bars + 8 * (B_V_EMPTY + s));
+        }
+        __syncwarp();
+        ++pv_done[t];
+        // Tile 0 done one block before the unit ends: issue the next unit's
+        // first S_0 now (as for pair units below).
+        if (t == 0 && !s0_pre && u_next >= 0 && idx + 2 == U.n_iter) {
+          const uint32_t it2 = kv_it + U.n_iter;
+          const int s2 = it2 % NUM_STAGES;
+          ok = warp_wait(bars + 8 * (B_K_FULL + s2), (it2 / NUM_STAGES) & 1u, abort_flag, p);
+          if (!ok) break;
+          ok = wait_q(q_slot(ul + 1, 0));
+          if (!ok) break;
+          if (elect_one()) {
+            issue_qk<D, BF16>(tmem, sbase, 0, q_slot(ul + 1, 0), s2);
+            mma_commit(bars + 8 * (B_S_FULL + 0));
+          }
+          __syncwarp();
+          ++n_s;
+          s0_pre = true;
+        }
+      }
+      kv_it += U.n_iter;
+      ++ul;
+      continue;
+    }
     for (int idx = 0; idx < U.n_iter && ok; ++idx) {
       const int j = block_at<REV>(U, idx);
       const uint32_t it = kv_it + idx;
@@ -546,7 +654,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       const uint32_t itn = it + 1;
       const int sn = itn % NUM_STAGES;
       // Q tile 0: P0 V_j, then S0 for the next block
-      if (tile_uses(U, 0, j)) {
+      if (tile_uses<SPLIT>(U, 0, j)) {
         ok = warp_wait(bars + 8 * (B_P_FULL + 0), p_ph[0], abort_flag, p);
         if (!ok) break;
         p_ph[0] ^= 1u;
@@ -562,7 +670,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         ok = warp_wait(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
         if (!ok) break;
         tc_fence_after_sync();
-        if (tile_uses(U, 0, jn)) {
+        if (tile_uses<SPLIT>(U, 0, jn)) {
           ok = need_q(0);
           if (!ok) break;
           if (elect_one()) {
@@ -574,7 +682,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         }
       }
       // Q tile 1: P1 V_j, then S1 for the next block
-      if (tile_uses(U, 1, j)) {
+      if (tile_uses<SPLIT>(U, 1, j)) {
         ok = warp_wait(bars + 8 * (B_P_FULL + 1), p_ph[1], abort_flag, p);
         if (!ok) break;
         p_ph[1] ^= 1u;
@@ -586,14 +694,14 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         __syncwarp();
         ++pv_done[1];
       }
-      if (has_next && tile_uses(U, 1, jn)) {
+      if (has_next && tile_uses<SPLIT>(U, 1, jn)) {
         ok = need_q(1);
         if (!ok) break;
       }
       if (elect_one()) {
         mma_commit(bars + 8 * (B_V_EMPTY + s));
         if (has_next) {
-          if (tile_uses(U, 1, jn)) {
+          if (tile_uses<SPLIT>(U, 1, jn)) {
             issue_qk<D, BF16>(tmem, sbase, 1, qs1, sn);
             mma_commit(bars + 8 * (B_S_FULL + 1));
           }
@@ -606,16 +714,16 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         }
       }
       __syncwarp();
-      if (has_next && tile_uses(U, 1, jn)) ++n_s;
+      if (has_next && tile_uses<SPLIT>(U, 1, jn)) ++n_s;
       // Once Q tile 0 has no block left in this unit (its last P_0 V is
       // issued and no S_0 follows), its next S is the next unit's first one:
       // issue it now, so that softmax 0 finds it ready after its epilogue
       // instead of waiting for tile 1 to finish this unit.  S_0 overwrites
       // P_0 only after the P_0 V issued before it (the pipe runs in order).
-      if (!s0_pre && u_next >= 0 && has_next && !tile_uses(U, 0, jn) && idx + 2 == U.n_iter) {
-        const Unit UN = decode_unit<REV>(u_next, p);
+      if (!s0_pre && u_next >= 0 && has_next && !tile_uses<SPLIT>(U, 0, jn) && idx + 2 == U.n_iter) {
+        const Unit UN = decode_unit<REV, SPLIT>(u_next, p);
         const int jn0 = block_at<REV>(UN, 0);
-        if (tile_uses(UN, 0, jn0)) {
+        if (tile_uses<SPLIT>(UN, 0, jn0)) {
           const uint32_t it2 = kv_it + U.n_iter;       // ring position of the next unit's first K
           const int s2 = it2 % NUM_STAGES;
           ok = warp_wait(bars + 8 * (B_K_FULL + s2), (it2 / NUM_STAGES) & 1u, abort_flag, p);
@@ -645,7 +753,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   drain_wait(bars + 8 * B_DRAIN, 0, p.watchdog_ns);
 }
 
-template <int D, bool BF16, bool OUT_F32, bool ALIBI>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI, bool SPLIT>
 __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint32_t tmem,
                              uint32_t sbase, uint32_t bars, int t, int warp_in_wg, int lane,
                              volatile int* abort_flag) {
@@ -655,11 +763,14 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
   const uint32_t lane_base = static_cast<uint32_t>(warp_in_wg * 32) << 16;
   const uint32_t s_tmem = tmem + lane_base + G::S_COL0 + t * BN;
   const uint32_t o_tmem = tmem + lane_base + G::O_COL0 + t * D;
+  const uint32_t o1_tmem = tmem + lane_base + G::O_COL0 + D;   // split units: the other half's O
+  // split units: warpgroup 1's (m, l_exact, l_round) for each row
+  const uint32_t half_stats = sbase + G::STATS_OFF + 12 * row_in_tile;
   const float c = p.scale_log2;
   // 16-bit output rows of 128 bytes per 64-column chunk are staged in shared
   // memory and written by TMA; other outputs are stored from registers.
   constexpr bool STAGED = !OUT_F32 && G::CB == 128;
-  uint32_t s_ph = 0, o_ph = 0, epi_ph = 0;
+  uint32_t s_ph = 0, o_ph = 0, epi_ph = 0, half_ph = 0, o1_ph = 0;
   bool ok = true;
   int ul = -1;
   // Q_EMPTY barrier of the slot whose staged output a TMA store issued by
@@ -678,9 +789,15 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     ++ul;
-    const Unit U = decode_unit<ALIBI>(u, p);
-    if (t >= U.n_active) continue;
-    const int r0 = U.q0 + t * BM;
+    const Unit U = decode_unit<ALIBI, SPLIT>(u, p);
+    if (!SPLIT && t >= U.n_active) continue;
+    const int r0 = U.q0 + (SPLIT ? 0 : t * BM);
+    if (SPLIT && t == 1 && ul > 0) {
+      // O_1 and the row statistics of the CTA's previous unit must have been
+      // read by warpgroup 0 before this unit's first P_1 V overwrites O_1
+      ok = warp_wait(bars + 8 * B_HALF_FREE, (ul - 1) & 1u, abort_flag, p);
+      if (!ok) break;
+    }
     const int row = r0 + row_in_tile;
     // ALiBi slope of this query head in log2 units (the logits are kept in
     // units of log2 so that exp2 can be used)
@@ -689,7 +806,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     bool first = true;
     for (int idx = 0; idx < U.n_iter; ++idx) {
       const int j = block_at<ALIBI>(U, idx);
-      if (!tile_uses(U, t, j)) continue;
+      if (!tile_uses<SPLIT>(U, t, j)) continue;
       release_stage();
       // one verdict for the whole warp: the TMEM load and the vote below are
       // warp-collective, so no lane may leave the loop alone
@@ -871,12 +988,49 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       first = false;
     }
     if (!ok) break;
+    if (SPLIT && t == 1) {
+      // hand this half's row statistics to warpgroup 0, which merges
+      st_shared_f32(half_stats, m_run);
+      st_shared_f32(half_stats + 4, l_exact);
+      st_shared_f32(half_stats + 8, l_round);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * B_HALF);
+      continue;
+    }
     // epilogue: O = O_acc / l, written once; LSE = (m + log2 l) ln 2
     ok = warp_wait(bars + 8 * (B_O_FULL + t), o_ph, abort_flag, p);
     if (!ok) break;
     o_ph ^= 1u;
     tc_fence_after_sync();
+    // Split units: merge warpgroup 1's half, (m1, l1, O_1), into this one:
+    // m = max(m0, m1), each half weighted by exp2(m_half - m).
+    float w0 = 1.f, w1 = 0.f;
+    bool has1 = false;
+    if constexpr (SPLIT) {
+      ok = warp_wait(bars + 8 * B_HALF, half_ph, abort_flag, p);
+      if (!ok) break;
+      half_ph ^= 1u;
+      has1 = U.last1 >= 0;   // O_1 holds a sum only when warpgroup 1 visited a block
+      if (has1) {
+        ok = warp_wait(bars + 8 * (B_O_FULL + 1), o1_ph, abort_flag, p);
+        if (!ok) break;
+        o1_ph ^= 1u;
+        tc_fence_after_sync();
+      }
+      const float m1 = ld_shared_f32(half_stats), le1 = ld_shared_f32(half_stats + 4),
+                  lr1 = ld_shared_f32(half_stats + 8);
+      const float m = fmaxf(m_run, m1);
+      w0 = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m);
+      w1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - m);
+      l_exact = l_exact * w0 + le1 * w1;
+      l_round = l_round * w0 + lr1 * w1;
+      m_run = m;
+    }
     const float inv_l = 1.f / l_round;
+    w0 *= inv_l;
+    w1 *= inv_l;
+    // the per-element scale of O_0 (split units fold it into the merge below)
+    const float sc = SPLIT ? 1.f : inv_l;
     const bool valid = row < p.N;
     const uint32_t q_empty = bars + 8 * (B_Q_EMPTY + q_slot(ul, t));
     if constexpr (STAGED) {
@@ -891,11 +1045,11 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t orr[32];
         tmem_ld_32x32b_x32(o_tmem + cc * 32, orr);
+        if constexpr (SPLIT) merge_half<32>(orr, o1_tmem + cc * 32, has1, w0, w1);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pk[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
-                              __uint_as_float(orr[2 * e + 1]) * inv_l);
+          pk[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * sc, __uint_as_float(orr[2 * e + 1]) * sc);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int unit = (cc & 1) * 4 + k4;   // 16-byte unit within the 128-byte row
@@ -925,22 +1079,23 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       for (int cc = 0; cc < D / OC; ++cc) {
         uint32_t orr[OC];
         tmem_ld_cols<OC>(o_tmem + cc * OC, orr);
+        if constexpr (SPLIT) merge_half<OC>(orr, o1_tmem + cc * OC, has1, w0, w1);
         if (valid) {
           if constexpr (OUT_F32) {
             float* dst = reinterpret_cast<float*>(p.o) + row_off + cc * OC;
 #pragma unroll
             for (int e = 0; e < OC; e += 4) {
               const float4 v4 = make_float4(
-                  __uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l,
-                  __uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
+                  __uint_as_float(orr[e]) * sc, __uint_as_float(orr[e + 1]) * sc,
+                  __uint_as_float(orr[e + 2]) * sc, __uint_as_float(orr[e + 3]) * sc);
               *reinterpret_cast<float4*>(dst + e) = v4;
             }
           } else {
             uint32_t packed[OC / 2];
 #pragma unroll
             for (int e = 0; e < OC / 2; ++e)
-              packed[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * inv_l,
-                                      __uint_as_float(orr[2 * e + 1]) * inv_l);
+              packed[e] = pack2<BF16>(__uint_as_float(orr[2 * e]) * sc,
+                                      __uint_as_float(orr[2 * e + 1]) * sc);
             uint16_t* dst = reinterpret_cast<uint16_t*>(p.o) + row_off + cc * OC;
 #pragma unroll
             for (int e = 0; e < OC / 2; e += 4)
@@ -951,6 +1106,12 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       }
       // the slot was not used for staging
       if (warp_in_wg == 0 && lane == 0) mbar_arrive(q_empty);
+    }
+    if constexpr (SPLIT) {
+      // O_1 and the statistics are read: warpgroup 1 may start its next unit
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * B_HALF_FREE);
     }
     if (valid && p.lse != nullptr)
       p.lse[static_cast<size_t>(U.bh) * p.N + row] = (m_run + __log2f(l_exact)) * 0.69314718055994531f;
@@ -965,7 +1126,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
   }
 }
 
-template <int D, bool BF16, bool OUT_F32, bool ALIBI>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -1004,6 +1165,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(bars + 8 * B_DRAIN, 1);
     mbar_init(bars + 8 * (B_EPI + 0), 4);   // one arrival per softmax warp
     mbar_init(bars + 8 * (B_EPI + 1), 4);
+    mbar_init(bars + 8 * B_HALF, 4);        // one arrival per softmax warp of warpgroup 1
+    mbar_init(bars + 8 * B_HALF_FREE, 4);   // one arrival per softmax warp of warpgroup 0
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -1031,16 +1194,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // smaller one.
   if (warp < 8) {
     regs_increase<SOFTMAX_REGS>();
-    softmax_role<D, BF16, OUT_F32, ALIBI>(p, &tmO, tmem, sbase, bars, warp / 4, warp % 4, lane,
+    softmax_role<D, BF16, OUT_F32, ALIBI, SPLIT>(p, &tmO, tmem, sbase, bars, warp / 4, warp % 4, lane,
                                           abort_flag);
     tc_fence_before_sync();
     __syncthreads();
   } else {
     regs_decrease<CONTROL_REGS>();
     if (warp == MMA_WARP) {
-      mma_role<D, BF16, ALIBI>(p, tmem, sbase, bars, abort_flag);
+      mma_role<D, BF16, ALIBI, SPLIT>(p, tmem, sbase, bars, abort_flag);
     } else if (warp == TMA_WARP) {
-      tma_role<D, ALIBI>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
+      tma_role<D, ALIBI, SPLIT>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();

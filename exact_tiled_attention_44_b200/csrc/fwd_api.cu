@@ -4,10 +4,17 @@
 
 namespace attn_host {
 
-// attn_fwd with an optional slope array (NULL: no position bias).
+bool fwd_split_units(int B, int H, int N, bool alibi, int sm_count) {
+  if (alibi) return false;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long pairs = bh * ((N + 2 * attn::BM - 1) / (2 * attn::BM));
+  const long long tiles = bh * ((N + attn::BM - 1) / attn::BM);
+  return pairs < sm_count && tiles <= 2LL * sm_count;
+}
+
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
              const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
-             int n_sink, float scale, int dtype, void* stream) {
+             int n_sink, float scale, int dtype, void* stream, int split) {
   Sizes sz;
   bool empty = false;
   int rc = validate(q, k, v, o, lse, B, H, H_kv, N, d, causal, window, n_sink, scale, dtype, &sz,
@@ -45,19 +52,23 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
   kp.window = (window >= N) ? 0 : window;
   kp.n_sink = kp.window > 0 ? (n_sink < N ? n_sink : N) : 0;
   kp.scale_log2 = scale * 1.4426950408889634f;
+  if (split < 0) split = g_force_units.load();
+  const bool sp = slopes == nullptr &&
+                  (split >= 0 ? split != 0 : fwd_split_units(B, H, N, false, st->sm_count));
   kp.n_qpairs = (N + 2 * attn::BM - 1) / (2 * attn::BM);
+  kp.n_qtiles = (N + attn::BM - 1) / attn::BM;
   kp.n_kblocks = (N + attn::BN - 1) / attn::BN;
-  kp.num_units = B * H * kp.n_qpairs;
+  kp.num_units = B * H * (sp ? kp.n_qtiles : kp.n_qpairs);
   kp.alibi = slopes;
   kp.withhold_loads = take_withhold();
   kp.block_count = g_block_count.load();
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 16: return launch_d<16>(st, bf16, f32, mq, mk, mv, mo, kp, s);
-    case 32: return launch_d<32>(st, bf16, f32, mq, mk, mv, mo, kp, s);
-    case 64: return launch_d<64>(st, bf16, f32, mq, mk, mv, mo, kp, s);
-    case 128: return launch_fwd_d128(st, bf16, f32, mq, mk, mv, mo, kp, s);
+    case 16: return launch_d<16>(st, bf16, f32, sp, mq, mk, mv, mo, kp, s);
+    case 32: return launch_d<32>(st, bf16, f32, sp, mq, mk, mv, mo, kp, s);
+    case 64: return launch_d<64>(st, bf16, f32, sp, mq, mk, mv, mo, kp, s);
+    case 128: return launch_fwd_d128(st, bf16, f32, sp, mq, mk, mv, mo, kp, s);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }

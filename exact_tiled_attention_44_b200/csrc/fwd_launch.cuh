@@ -7,18 +7,18 @@
 
 namespace attn_host {
 
-template <int D, bool BF16, bool F32, bool ALIBI>
+template <int D, bool BF16, bool F32, bool ALIBI, bool SPLIT>
 int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
                const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
                cudaStream_t stream) {
-  auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI>;
+  auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI, SPLIT>;
   // At least half of the SM's shared memory, so that two CTAs can never share
   // an SM (each allocates all 512 TMEM columns).
   const int smem_need = attn::Geo<D>::SMEM_BYTES + 1024;
   const int smem = smem_need > 120 * 1024 ? smem_need : 120 * 1024;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!(st->attr_set & (1u << bit))) {
+    if (!(st->attr_set & (1ull << bit))) {
       // The kernel re-splits its registers between warpgroups after launch;
       // that only works when every thread starts with LAUNCH_REGS registers.
       cudaFuncAttributes fa;
@@ -26,7 +26,7 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
       if (fa.numRegs < attn::LAUNCH_REGS) return ATTN_ERR_UNSUPPORTED;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return ATTN_ERR_CUDA;
-      st->attr_set |= 1u << bit;
+      st->attr_set |= 1ull << bit;
     }
   }
   const int grid = kp.num_units < st->sm_count ? kp.num_units : st->sm_count;
@@ -35,29 +35,32 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool ALIBI>
+template <int D, bool ALIBI, bool SPLIT>
 int launch_da(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
               const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
               cudaStream_t stream) {
   const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
-  const int bit = dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
+  const int bit = (SPLIT ? 32 : 0) + dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
   if (bf16)
-    return f32 ? launch_one<D, true, true, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream)
-               : launch_one<D, true, false, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream);
-  return f32 ? launch_one<D, false, true, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream)
-             : launch_one<D, false, false, ALIBI>(st, bit, mq, mk, mv, mo, kp, stream);
+    return f32 ? launch_one<D, true, true, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream)
+               : launch_one<D, true, false, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream);
+  return f32 ? launch_one<D, false, true, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream)
+             : launch_one<D, false, false, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream);
 }
 
+// `split`: one Q tile per unit, its key blocks shared out between the two
+// softmax warpgroups (no position bias); otherwise pairs of Q tiles.
 template <int D>
-int launch_d(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
-             const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
-             cudaStream_t stream) {
-  return kp.alibi != nullptr ? launch_da<D, true>(st, bf16, f32, mq, mk, mv, mo, kp, stream)
-                             : launch_da<D, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+int launch_d(DeviceState* st, bool bf16, bool f32, bool split, const CUtensorMap& mq,
+             const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+             const attn::KernelParams& kp, cudaStream_t stream) {
+  if (kp.alibi != nullptr) return launch_da<D, true, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+  return split ? launch_da<D, false, true>(st, bf16, f32, mq, mk, mv, mo, kp, stream)
+               : launch_da<D, false, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
 }
 
 // The d = 128 instantiations (compiled in their own translation unit).
-int launch_fwd_d128(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq,
+int launch_fwd_d128(DeviceState* st, bool bf16, bool f32, bool split, const CUtensorMap& mq,
                     const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                     const attn::KernelParams& kp, cudaStream_t stream);
 

@@ -27,7 +27,7 @@ struct DeviceState {
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
   int* status = nullptr;           // device address of the status word
-  uint32_t attr_set = 0;           // one bit per forward kernel instantiation
+  uint64_t attr_set = 0;           // one bit per forward kernel instantiation
   uint32_t dec_attr_set = 0;       // one bit per decode kernel instantiation
   uint32_t dec_small_attr_set = 0; // one bit per small-group decode kernel instantiation
   uint32_t bwd_attr_set = 0;       // one bit per backward kernel instantiation
@@ -44,6 +44,7 @@ extern std::atomic<unsigned long long> g_watchdog_ns;
 extern std::atomic<unsigned long long> g_launches;
 extern std::atomic<int> g_withhold;     // launches left that withhold their loads (test hook)
 extern std::atomic<unsigned long long*> g_block_count;   // block-count test hook (or nullptr)
+extern std::atomic<int> g_force_units;  // work-unit shape test hook: -1 automatic, 0 pairs, 1 split
 extern std::mutex g_host_mu;            // attn_fwd_host's streams and events
 extern PFN_cuTensorMapEncodeTiled_v12000 g_encode;
 
@@ -100,9 +101,17 @@ cudaError_t launch_overlapped(void (*kern)(Params...), int grid, int block, size
 // Takes one launch from the withhold-loads test hook, if any is pending.
 int take_withhold();
 
-// attn_fwd with an optional slope array (NULL: no position bias).
+// True when the forward runs one Q tile per work unit, its key blocks shared
+// out between the two softmax warpgroups: when pairs of Q tiles would leave
+// SMs idle and single tiles still fit about two waves (no position bias).
+bool fwd_split_units(int B, int H, int N, bool alibi, int sm_count);
+
+// attn_fwd with an optional slope array (NULL: no position bias).  split:
+// 1 / 0 forces split or pair units, -1 lets fwd_split_units decide (callers
+// that cut one problem into several launches pass the whole problem's choice,
+// so that every row is computed as the uncut call computes it).
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
              const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
-             int n_sink, float scale, int dtype, void* stream);
+             int n_sink, float scale, int dtype, void* stream, int split = -1);
 
 }  // namespace attn_host

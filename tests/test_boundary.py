@@ -187,6 +187,13 @@ def test_withhold_hook_arguments():
     assert A.test_withhold_loads(0) == A.ATTN_OK
 
 
+def test_force_units_hook_arguments():
+    for bad in (-2, 2, 7):
+        assert A.test_force_units(bad) == A.ATTN_ERR_INVALID_ARG
+    for mode in (0, 1, -1):
+        assert A.test_force_units(mode) == A.ATTN_OK
+
+
 def test_count_blocks_hook_arguments():
     assert A.test_count_blocks(None) == A.ATTN_OK
     with pytest.raises(ValueError):

@@ -65,6 +65,54 @@ def test_sweep_full_parity(case):
     assert torch.equal(l16, l32)
 
 
+@pytest.fixture
+def units():
+    """Runs a test under a forced work-unit shape and restores the automatic choice."""
+    def force(mode):
+        assert A.test_force_units(mode) == A.ATTN_OK
+    yield force
+    A.test_force_units(-1)
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["pairs", "split"])
+@pytest.mark.parametrize("case", SWEEP, ids=[_id(c) for c in SWEEP])
+def test_sweep_both_unit_shapes(case, mode, units):
+    """Every sweep case with pairs of Q tiles and with single Q tiles whose key
+    blocks the two softmax warpgroups share (the automatic choice takes one of
+    them by problem size): both against the oracle, the 16-bit output the fp32
+    one rounded once."""
+    units(mode)
+    B, H, Hk, N, d, dt, causal, window, n_sink = case
+    q, k, v = random_qkv(B, H, Hk, N, d, dt, seed=N * 131 + d)
+    scale = A.default_scale(d)
+    Or, Lr = oracle_full(q, k, v, bool(causal), window, n_sink, scale)
+    o32, l32 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=True)
+    assert_parity(errors(o32, l32, Or, Lr), what="fp32 out")
+    o16, l16 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=False)
+    assert_parity(errors(o16, l16, Or, Lr), round_floor(Or, dt), what="16-bit out")
+    assert torch.equal(o16, o32.to(dt)) and torch.equal(l16, l32)
+    assert A.get_status() == A.ATTN_OK
+
+
+@pytest.mark.parametrize("wl", ["c2", "c2c"])
+def test_small_workloads_split_units_against_oracle_and_pairs(wl, units):
+    """c2 / c2c in full run as split units by default; they match the oracle
+    and the pair-unit result to the fp32 rounding level."""
+    w = WORKLOADS[wl]
+    q, k, v = make_inputs(w)
+    Or, Lr = oracle_full(q, k, v, w.causal, w.window, w.n_sink, w.scale)
+    units(1)
+    o1, l1 = run_gpu(q, k, v, w.causal, w.window, w.n_sink, w.scale, out_f32=True)
+    units(0)
+    o0, l0 = run_gpu(q, k, v, w.causal, w.window, w.n_sink, w.scale, out_f32=True)
+    units(-1)
+    oa, la = run_gpu(q, k, v, w.causal, w.window, w.n_sink, w.scale, out_f32=True)
+    assert torch.equal(oa, o1) and torch.equal(la, l1)       # the automatic choice is split
+    assert_parity(errors(o1, l1, Or, Lr), what="split units")
+    assert_parity(errors(o0, l0, Or, Lr), what="pair units")
+    assert (o1 - o0).abs().max().item() < 1e-2 and (l1 - l0).abs().max().item() < 1e-5
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.2, 0.9, 3.0])
 def test_scale_values(scale):
     q, k, v = random_qkv(1, 2, 2, 300, 64, BF, seed=7)

@@ -47,6 +47,22 @@ def test_forward_computes_exactly_the_visited_blocks(case):
     assert got == A.visited_blocks(N, bool(causal), window, n_sink) * B * H
 
 
+@pytest.mark.parametrize("mode", [0, 1], ids=["pairs", "split"])
+@pytest.mark.parametrize("case", CASES)
+def test_forward_unit_shapes_compute_exactly_the_visited_blocks(case, mode):
+    """Pairs of Q tiles and single Q tiles shared by both softmax warpgroups
+    compute the same set of score tiles."""
+    B, H, H_kv, N, d, dt, causal, window, n_sink = case
+    q, k, v = (t.cuda() for t in random_qkv(B, H, H_kv, N, d, dt, seed=1))
+    assert A.test_force_units(mode) == A.ATTN_OK
+    try:
+        got = _count(lambda: A.attention(q, k, v, causal=bool(causal), window=window,
+                                         n_sink=n_sink))
+    finally:
+        A.test_force_units(-1)
+    assert got == A.visited_blocks(N, bool(causal), window, n_sink) * B * H
+
+
 @pytest.mark.parametrize("case", CASES)
 def test_forward_with_position_bias_computes_exactly_the_visited_blocks(case):
     """With ALiBi slopes the forward walks every unit's blocks in descending
