@@ -146,8 +146,8 @@ def test_withhold_loads(n_launches: int) -> int:
 
 def test_force_units(mode: int) -> int:
     """Work-unit shape hook for tests: 0 forces pairs of Q tiles, 1 single
-    tiles shared by both softmax warpgroups, -1 the automatic choice (see
-    include/attn.h)."""
+    tiles shared by both softmax warpgroups, 2 pairs of query heads sharing a
+    K/V head, -1 the automatic choice (see include/attn.h)."""
     return int(load_library().attn_test_force_units(int(mode)))
 
 

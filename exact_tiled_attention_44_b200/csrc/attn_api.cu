@@ -176,7 +176,7 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   const int G = H / H_kv;
   // every chunk runs the work-unit shape attn_fwd would choose for the whole problem
   const int forced = g_force_units.load();
-  const bool split = forced >= 0 ? forced == 1 : fwd_split_units(B, H, N, false, st->sm_count);
+  const int uk = forced >= 0 ? forced : fwd_unit_kind(B, H, H_kv, N, window, false, st->sm_count);
   // chunked LSE rows must keep the 16-byte alignment attn_fwd requires
   const bool lse_ok = !with_lse || (static_cast<long long>(G) * N) % 4 == 0;
   const int n_chunks = lse_ok ? static_cast<int>(groups < kHostChunks ? groups : kHostChunks) : 1;
@@ -218,7 +218,7 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
         cudaEventRecord(in, st->copy_in) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess)
       return ATTN_ERR_CUDA;
     rc = fwd_impl(dqc, dkc, dvc, doc, dlc, nullptr, static_cast<int>(T), G, 1, N, d, causal, window,
-                  n_sink, scale, dtype, stream, split ? 1 : 0);
+                  n_sink, scale, dtype, stream, uk);
     if (rc != ATTN_OK) return rc;
     if (cudaEventRecord(out, s) != cudaSuccess || cudaStreamWaitEvent(st->copy_out, out, 0) != cudaSuccess ||
         cudaMemcpyAsync(const_cast<char*>(at(o, g0 * o_grp)), doc, T * o_grp, cudaMemcpyDeviceToHost,
@@ -321,7 +321,7 @@ int attn_test_count_blocks(unsigned long long* counter) {
 }
 
 int attn_test_force_units(int mode) {
-  if (mode < -1 || mode > 1) return ATTN_ERR_INVALID_ARG;
+  if (mode < -1 || mode > 2) return ATTN_ERR_INVALID_ARG;
   g_force_units.store(mode);
   return ATTN_OK;
 }

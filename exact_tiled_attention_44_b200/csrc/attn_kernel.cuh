@@ -41,6 +41,7 @@
 
 namespace attn {
 
+constexpr int UK_PAIR = 0, UK_SPLIT = 1, UK_HEADS = 2;   // work-unit kinds (see decode_unit)
 constexpr int BM = 128;           // query rows per Q tile
 constexpr int BN = 128;           // keys per K/V block
 constexpr int NUM_STAGES = 2;     // K ring depth (and V ring depth)
@@ -72,8 +73,10 @@ struct KernelParams {
   float scale_log2;   // scale * log2(e)
   int n_qpairs;       // ceil(N / 256)
   int n_qtiles;       // ceil(N / 128)
+  int n_hpairs;       // ceil(G / 2): pairs of query heads of one K/V head (G = H / H_kv)
   int n_kblocks;      // ceil(N / 128)
-  int num_units;      // B * H * n_qpairs (pair units) or B * H * n_qtiles (split units)
+  int num_units;      // B * H * n_qpairs (pair units), B * H * n_qtiles (split units)
+                      // or B * H_kv * n_hpairs * n_qtiles (head-pair units)
   const float* alibi; // ALiBi slope per query head ([H], device), used by the ALIBI kernels
   int withhold_loads; // test hook: the TMA warp issues nothing, so every wait runs out
   unsigned long long* block_count;  // test hook: S tiles computed are added here (or nullptr)
@@ -168,30 +171,51 @@ struct Unit {
 // position bias: the bias grows towards the diagonal, so the nearest keys come
 // first and the running row max seldom has to move (each move rescales O).
 //
-// SPLIT: a unit is one Q tile instead of a pair, and the two softmax
-// warpgroups ("tiles" t = 0, 1 below) share its rows: t takes the visited
-// blocks at even (t = 0) or odd (t = 1) positions, with its own S_t, O_t and
-// running (m, l); warpgroup 0 merges the halves in the epilogue.  Used when
-// pair units would leave SMs idle (few heads, short sequences).
-template <bool REV, bool SPLIT>
+// UK, the unit kind:
+//   UK_PAIR  two consecutive 128-row Q tiles of one head (t = 0, 1);
+//   UK_SPLIT one Q tile, and the two softmax warpgroups ("tiles" t = 0, 1
+//            below) share its rows: t takes the visited blocks at even (t = 0)
+//            or odd (t = 1) positions, with its own S_t, O_t and running
+//            (m, l); warpgroup 0 merges the halves in the epilogue.  Used when
+//            pair units would leave SMs idle (few heads, short sequences);
+//   UK_HEADS the same 128 rows of two query heads h, h + 1 that share one K/V
+//            head (GQA / MQA): every K/V block loaded feeds both tiles.
+template <bool REV, int UK>
 __device__ __forceinline__ Unit decode_unit(int u, const KernelParams& p) {
+  constexpr bool SPLIT = UK == UK_SPLIT, HEADS = UK == UK_HEADS;
   static_assert(!(REV && SPLIT), "split units visit blocks in ascending order");
   Unit U;
-  const int BH = p.B * p.H;
-  // Longest-processing-time first: causal cost grows with the pair (tile)
-  // index, so units are handed out from the last pair of every head down.
-  const int pair = (SPLIT ? p.n_qtiles : p.n_qpairs) - 1 - u / BH;
-  U.bh = u % BH;
-  U.b = U.bh / p.H;
-  U.h = U.bh % p.H;
-  U.g = U.h / (p.H / p.H_kv);
-  U.q0 = pair * (SPLIT ? 1 : 2) * BM;
-  U.n_active = (!SPLIT && U.q0 + BM < p.N) ? 2 : 1;
+  if constexpr (HEADS) {
+    // Longest first by row position; within one, the head pairs of a K/V
+    // head are adjacent, so the CTAs in flight share K/V blocks in L2.
+    const int per_pos = p.B * p.H_kv * p.n_hpairs;
+    const int pos = p.n_qtiles - 1 - u / per_pos;
+    const int rem = u % per_pos;
+    const int G = p.H / p.H_kv;
+    U.b = rem / (p.H_kv * p.n_hpairs);
+    U.g = (rem / p.n_hpairs) % p.H_kv;
+    const int hp = rem % p.n_hpairs;
+    U.h = U.g * G + 2 * hp;
+    U.bh = U.b * p.H + U.h;
+    U.q0 = pos * BM;
+    U.n_active = (2 * hp + 1 < G) ? 2 : 1;
+  } else {
+    const int BH = p.B * p.H;
+    // Longest-processing-time first: causal cost grows with the pair (tile)
+    // index, so units are handed out from the last pair of every head down.
+    const int pair = (SPLIT ? p.n_qtiles : p.n_qpairs) - 1 - u / BH;
+    U.bh = u % BH;
+    U.b = U.bh / p.H;
+    U.h = U.bh % p.H;
+    U.g = U.h / (p.H / p.H_kv);
+    U.q0 = pair * (SPLIT ? 1 : 2) * BM;
+    U.n_active = (!SPLIT && U.q0 + BM < p.N) ? 2 : 1;
+  }
   const int sink_blocks = (p.window > 0) ? (p.n_sink + BN - 1) / BN : 0;
   int sb = 0, lo_min = 1 << 30, hi_max = 0;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int r0 = U.q0 + (SPLIT ? 0 : t * BM);
+    const int r0 = U.q0 + (UK == UK_PAIR ? t * BM : 0);
     const int r_last = min(r0 + BM - 1, p.N - 1);
     int lo = 0, hi = p.n_kblocks;
     if (p.causal) hi = min(p.n_kblocks, r_last / BN + 1);
@@ -254,9 +278,20 @@ __device__ __forceinline__ int block_at(const Unit& U, int idx) {
   return k < U.sb ? k : U.wlo + (k - U.sb);
 }
 
-template <bool SPLIT>
+// First query row and (batch, head) index of tile t's rows.
+template <int UK>
+__device__ __forceinline__ int tile_row0_k(const Unit& U, int t) {
+  return U.q0 + (UK == UK_PAIR ? t * BM : 0);
+}
+
+template <int UK>
+__device__ __forceinline__ int tile_bh_k(const Unit& U, int t) {
+  return U.bh + (UK == UK_HEADS ? t : 0);
+}
+
+template <int UK>
 __device__ __forceinline__ bool tile_uses(const Unit& U, int t, int j) {
-  if constexpr (SPLIT) {
+  if constexpr (UK == UK_SPLIT) {
     const int idx = j < U.sb ? j : U.sb + (j - U.wlo);   // position of visited block j
     return (idx & 1) == t;
   }
@@ -386,7 +421,7 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)
 
 // ------------------------------------------------------------ roles
 
-template <int D, bool REV, bool SPLIT>
+template <int D, bool REV, int UK>
 __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                          const CUtensorMap* tmV, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
@@ -410,7 +445,7 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
       mbar_arrive_expect_tx(bars + 8 * (B_Q_FULL + qs), G::TILE_BYTES);
       for (int c = 0; c < G::NCH; ++c)
         tma_load_3d(sbase + G::Q_OFF + qs * G::TILE_BYTES + c * G::CHUNK_BYTES, tmQ,
-                    bars + 8 * (B_Q_FULL + qs), c * G::CW, U.q0 + t * BM, U.bh);
+                    bars + 8 * (B_Q_FULL + qs), c * G::CW, tile_row0_k<UK>(U, t), tile_bh_k<UK>(U, t));
     }
     __syncwarp();
     q_last[qs] = static_cast<int>(ph);
@@ -422,7 +457,7 @@ __device__ void tma_role(const KernelParams& p, const CUtensorMap* tmQ, const CU
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit<REV, SPLIT>(u, p);
+    const Unit U = decode_unit<REV, UK>(u, p);
     // Loads in the order their ring stages and Q slots are released, so
     // that no load waits behind one whose slot frees later: Q tile 0 (its
     // slot was released by the unit before last), the first K block (whose
@@ -511,9 +546,10 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sbase, int t, i
   }
 }
 
-template <int D, bool BF16, bool REV, bool SPLIT>
+template <int D, bool BF16, bool REV, int UK>
 __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, uint32_t bars,
                          volatile int* abort_flag) {
+  constexpr bool SPLIT = UK == UK_SPLIT;
   uint32_t kv_it = 0, p_ph[2] = {0, 0};
   uint32_t q_uses[Q_SLOTS] = {0, 0, 0};
   unsigned long long n_s = 0;   // (Q tile, K/V block) score tiles issued, for the test hook
@@ -526,7 +562,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   for (int r = 0; r < rounds && ok; ++r) {
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
-    const Unit U = decode_unit<REV, SPLIT>(u, p);
+    const Unit U = decode_unit<REV, UK>(u, p);
     // split units: both tiles read the unit's one Q tile
     const int qs0 = q_slot(ul, 0), qs1 = SPLIT ? qs0 : q_slot(ul, 1);
     auto wait_q = [&](int qs) {
@@ -558,7 +594,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       if (!ok) break;
       tc_fence_after_sync();
       for (int t = 0; t < 2 && ok; ++t) {
-        if (!tile_uses<SPLIT>(U, t, j0)) continue;
+        if (!tile_uses<UK>(U, t, j0)) continue;
         if (t == 0 && this_s0_pre) continue;        // issued at the end of the unit before
         ok = need_q(t);
         if (!ok) break;
@@ -654,7 +690,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
       const uint32_t itn = it + 1;
       const int sn = itn % NUM_STAGES;
       // Q tile 0: P0 V_j, then S0 for the next block
-      if (tile_uses<SPLIT>(U, 0, j)) {
+      if (tile_uses<UK>(U, 0, j)) {
         ok = warp_wait(bars + 8 * (B_P_FULL + 0), p_ph[0], abort_flag, p);
         if (!ok) break;
         p_ph[0] ^= 1u;
@@ -670,7 +706,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         ok = warp_wait(bars + 8 * (B_K_FULL + sn), (itn / NUM_STAGES) & 1u, abort_flag, p);
         if (!ok) break;
         tc_fence_after_sync();
-        if (tile_uses<SPLIT>(U, 0, jn)) {
+        if (tile_uses<UK>(U, 0, jn)) {
           ok = need_q(0);
           if (!ok) break;
           if (elect_one()) {
@@ -682,7 +718,7 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         }
       }
       // Q tile 1: P1 V_j, then S1 for the next block
-      if (tile_uses<SPLIT>(U, 1, j)) {
+      if (tile_uses<UK>(U, 1, j)) {
         ok = warp_wait(bars + 8 * (B_P_FULL + 1), p_ph[1], abort_flag, p);
         if (!ok) break;
         p_ph[1] ^= 1u;
@@ -694,14 +730,14 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         __syncwarp();
         ++pv_done[1];
       }
-      if (has_next && tile_uses<SPLIT>(U, 1, jn)) {
+      if (has_next && tile_uses<UK>(U, 1, jn)) {
         ok = need_q(1);
         if (!ok) break;
       }
       if (elect_one()) {
         mma_commit(bars + 8 * (B_V_EMPTY + s));
         if (has_next) {
-          if (tile_uses<SPLIT>(U, 1, jn)) {
+          if (tile_uses<UK>(U, 1, jn)) {
             issue_qk<D, BF16>(tmem, sbase, 1, qs1, sn);
             mma_commit(bars + 8 * (B_S_FULL + 1));
           }
@@ -714,16 +750,16 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
         }
       }
       __syncwarp();
-      if (has_next && tile_uses<SPLIT>(U, 1, jn)) ++n_s;
+      if (has_next && tile_uses<UK>(U, 1, jn)) ++n_s;
       // Once Q tile 0 has no block left in this unit (its last P_0 V is
       // issued and no S_0 follows), its next S is the next unit's first one:
       // issue it now, so that softmax 0 finds it ready after its epilogue
       // instead of waiting for tile 1 to finish this unit.  S_0 overwrites
       // P_0 only after the P_0 V issued before it (the pipe runs in order).
-      if (!s0_pre && u_next >= 0 && has_next && !tile_uses<SPLIT>(U, 0, jn) && idx + 2 == U.n_iter) {
-        const Unit UN = decode_unit<REV, SPLIT>(u_next, p);
+      if (!s0_pre && u_next >= 0 && has_next && !tile_uses<UK>(U, 0, jn) && idx + 2 == U.n_iter) {
+        const Unit UN = decode_unit<REV, UK>(u_next, p);
         const int jn0 = block_at<REV>(UN, 0);
-        if (tile_uses<SPLIT>(UN, 0, jn0)) {
+        if (tile_uses<UK>(UN, 0, jn0)) {
           const uint32_t it2 = kv_it + U.n_iter;       // ring position of the next unit's first K
           const int s2 = it2 % NUM_STAGES;
           ok = warp_wait(bars + 8 * (B_K_FULL + s2), (it2 / NUM_STAGES) & 1u, abort_flag, p);
@@ -753,10 +789,11 @@ __device__ void mma_role(const KernelParams& p, uint32_t tmem, uint32_t sbase, u
   drain_wait(bars + 8 * B_DRAIN, 0, p.watchdog_ns);
 }
 
-template <int D, bool BF16, bool OUT_F32, bool ALIBI, bool SPLIT>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI, int UK>
 __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint32_t tmem,
                              uint32_t sbase, uint32_t bars, int t, int warp_in_wg, int lane,
                              volatile int* abort_flag) {
+  constexpr bool SPLIT = UK == UK_SPLIT;
   using G = Geo<D>;
   constexpr int OC = D >= 32 ? 32 : 16;   // TMEM columns per O load/store
   const int row_in_tile = warp_in_wg * 32 + lane;
@@ -789,9 +826,10 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     const int u = unit_of_round(r, blockIdx.x, gridDim.x, p.num_units);
     if (u < 0) continue;
     ++ul;
-    const Unit U = decode_unit<ALIBI, SPLIT>(u, p);
+    const Unit U = decode_unit<ALIBI, UK>(u, p);
     if (!SPLIT && t >= U.n_active) continue;
-    const int r0 = U.q0 + (SPLIT ? 0 : t * BM);
+    const int r0 = tile_row0_k<UK>(U, t);
+    const int bh = tile_bh_k<UK>(U, t);
     if (SPLIT && t == 1 && ul > 0) {
       // O_1 and the row statistics of the CTA's previous unit must have been
       // read by warpgroup 0 before this unit's first P_1 V overwrites O_1
@@ -801,12 +839,12 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
     const int row = r0 + row_in_tile;
     // ALiBi slope of this query head in log2 units (the logits are kept in
     // units of log2 so that exp2 can be used)
-    const float slope2 = ALIBI ? p.alibi[U.h] * 1.4426950408889634f : 0.f;
+    const float slope2 = ALIBI ? p.alibi[U.h + (UK == UK_HEADS ? t : 0)] * 1.4426950408889634f : 0.f;
     float m_run = -INFINITY, l_exact = 0.f, l_round = 0.f;
     bool first = true;
     for (int idx = 0; idx < U.n_iter; ++idx) {
       const int j = block_at<ALIBI>(U, idx);
-      if (!tile_uses<SPLIT>(U, t, j)) continue;
+      if (!tile_uses<UK>(U, t, j)) continue;
       release_stage();
       // one verdict for the whole warp: the TMEM load and the vote below are
       // warp-collective, so no lane may leave the loop alone
@@ -1065,7 +1103,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
         if (ok && lane == 0) {
 #pragma unroll
           for (int cch = 0; cch < G::NCH; ++cch)
-            tma_store_3d(tmO, stage + cch * G::CHUNK_BYTES, cch * G::CW, r0, U.bh);
+            tma_store_3d(tmO, stage + cch * G::CHUNK_BYTES, cch * G::CW, r0, bh);
           bulk_commit_group();
           // the slot is released once the store has read it (see release_stage)
           staged_slot = q_empty;
@@ -1074,7 +1112,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       }
       epi_ph ^= 1u;
     } else {
-      const size_t row_off = (static_cast<size_t>(U.bh) * p.N + row) * D;
+      const size_t row_off = (static_cast<size_t>(bh) * p.N + row) * D;
 #pragma unroll
       for (int cc = 0; cc < D / OC; ++cc) {
         uint32_t orr[OC];
@@ -1114,7 +1152,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       if (lane == 0) mbar_arrive(bars + 8 * B_HALF_FREE);
     }
     if (valid && p.lse != nullptr)
-      p.lse[static_cast<size_t>(U.bh) * p.N + row] = (m_run + __log2f(l_exact)) * 0.69314718055994531f;
+      p.lse[static_cast<size_t>(bh) * p.N + row] = (m_run + __log2f(l_exact)) * 0.69314718055994531f;
   }
   // the output stores this warp issued complete before the CTA can exit
   if (STAGED && warp_in_wg == 0) {
@@ -1126,7 +1164,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
   }
 }
 
-template <int D, bool BF16, bool OUT_F32, bool ALIBI, bool SPLIT>
+template <int D, bool BF16, bool OUT_F32, bool ALIBI, int UK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -1194,16 +1232,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // smaller one.
   if (warp < 8) {
     regs_increase<SOFTMAX_REGS>();
-    softmax_role<D, BF16, OUT_F32, ALIBI, SPLIT>(p, &tmO, tmem, sbase, bars, warp / 4, warp % 4, lane,
+    softmax_role<D, BF16, OUT_F32, ALIBI, UK>(p, &tmO, tmem, sbase, bars, warp / 4, warp % 4, lane,
                                           abort_flag);
     tc_fence_before_sync();
     __syncthreads();
   } else {
     regs_decrease<CONTROL_REGS>();
     if (warp == MMA_WARP) {
-      mma_role<D, BF16, ALIBI, SPLIT>(p, tmem, sbase, bars, abort_flag);
+      mma_role<D, BF16, ALIBI, UK>(p, tmem, sbase, bars, abort_flag);
     } else if (warp == TMA_WARP) {
-      tma_role<D, ALIBI, SPLIT>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
+      tma_role<D, ALIBI, UK>(p, &tmQ, &tmK, &tmV, sbase, bars, abort_flag);
     }
     tc_fence_before_sync();
     __syncthreads();

@@ -7,11 +7,11 @@
 
 namespace attn_host {
 
-template <int D, bool BF16, bool F32, bool ALIBI, bool SPLIT>
+template <int D, bool BF16, bool F32, bool ALIBI, int UK>
 int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMap& mk,
                const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
                cudaStream_t stream) {
-  auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI, SPLIT>;
+  auto kern = attn::attn_fwd_kernel<D, BF16, F32, ALIBI, UK>;
   // At least half of the SM's shared memory, so that two CTAs can never share
   // an SM (each allocates all 512 TMEM columns).
   const int smem_need = attn::Geo<D>::SMEM_BYTES + 1024;
@@ -35,32 +35,36 @@ int launch_one(DeviceState* st, int bit, const CUtensorMap& mq, const CUtensorMa
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <int D, bool ALIBI, bool SPLIT>
+template <int D, bool ALIBI, int UK>
 int launch_da(DeviceState* st, bool bf16, bool f32, const CUtensorMap& mq, const CUtensorMap& mk,
               const CUtensorMap& mv, const CUtensorMap& mo, const attn::KernelParams& kp,
               cudaStream_t stream) {
   const int dbit = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
-  const int bit = (SPLIT ? 32 : 0) + dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
+  const int bit = UK * 32 + dbit * 8 + (ALIBI ? 4 : 0) + (bf16 ? 2 : 0) + (f32 ? 1 : 0);
   if (bf16)
-    return f32 ? launch_one<D, true, true, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream)
-               : launch_one<D, true, false, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream);
-  return f32 ? launch_one<D, false, true, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream)
-             : launch_one<D, false, false, ALIBI, SPLIT>(st, bit, mq, mk, mv, mo, kp, stream);
+    return f32 ? launch_one<D, true, true, ALIBI, UK>(st, bit, mq, mk, mv, mo, kp, stream)
+               : launch_one<D, true, false, ALIBI, UK>(st, bit, mq, mk, mv, mo, kp, stream);
+  return f32 ? launch_one<D, false, true, ALIBI, UK>(st, bit, mq, mk, mv, mo, kp, stream)
+             : launch_one<D, false, false, ALIBI, UK>(st, bit, mq, mk, mv, mo, kp, stream);
 }
 
-// `split`: one Q tile per unit, its key blocks shared out between the two
-// softmax warpgroups (no position bias); otherwise pairs of Q tiles.
+// `uk`: the work-unit kind (attn::UK_PAIR, UK_SPLIT or UK_HEADS); launches
+// with a position bias always use pairs.
 template <int D>
-int launch_d(DeviceState* st, bool bf16, bool f32, bool split, const CUtensorMap& mq,
+int launch_d(DeviceState* st, bool bf16, bool f32, int uk, const CUtensorMap& mq,
              const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
              const attn::KernelParams& kp, cudaStream_t stream) {
-  if (kp.alibi != nullptr) return launch_da<D, true, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
-  return split ? launch_da<D, false, true>(st, bf16, f32, mq, mk, mv, mo, kp, stream)
-               : launch_da<D, false, false>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+  if (kp.alibi != nullptr)
+    return launch_da<D, true, attn::UK_PAIR>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+  if (uk == attn::UK_SPLIT)
+    return launch_da<D, false, attn::UK_SPLIT>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+  if (uk == attn::UK_HEADS)
+    return launch_da<D, false, attn::UK_HEADS>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
+  return launch_da<D, false, attn::UK_PAIR>(st, bf16, f32, mq, mk, mv, mo, kp, stream);
 }
 
 // The d = 128 instantiations (compiled in their own translation unit).
-int launch_fwd_d128(DeviceState* st, bool bf16, bool f32, bool split, const CUtensorMap& mq,
+int launch_fwd_d128(DeviceState* st, bool bf16, bool f32, int uk, const CUtensorMap& mq,
                     const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                     const attn::KernelParams& kp, cudaStream_t stream);
 

@@ -44,7 +44,7 @@ extern std::atomic<unsigned long long> g_watchdog_ns;
 extern std::atomic<unsigned long long> g_launches;
 extern std::atomic<int> g_withhold;     // launches left that withhold their loads (test hook)
 extern std::atomic<unsigned long long*> g_block_count;   // block-count test hook (or nullptr)
-extern std::atomic<int> g_force_units;  // work-unit shape test hook: -1 automatic, 0 pairs, 1 split
+extern std::atomic<int> g_force_units;  // work-unit kind test hook: -1 automatic, else attn::UK_*
 extern std::mutex g_host_mu;            // attn_fwd_host's streams and events
 extern PFN_cuTensorMapEncodeTiled_v12000 g_encode;
 
@@ -101,17 +101,19 @@ cudaError_t launch_overlapped(void (*kern)(Params...), int grid, int block, size
 // Takes one launch from the withhold-loads test hook, if any is pending.
 int take_withhold();
 
-// True when the forward runs one Q tile per work unit, its key blocks shared
-// out between the two softmax warpgroups: when pairs of Q tiles would leave
-// SMs idle and single tiles still fit about two waves (no position bias).
-bool fwd_split_units(int B, int H, int N, bool alibi, int sm_count);
+// The forward's work-unit kind (attn::UK_*): split units (one Q tile, its
+// key blocks shared out between the two softmax warpgroups) when pairs of Q
+// tiles would leave SMs idle and single tiles still fit about two waves; head
+// pairs for grouped heads whose rows see at most 4096 keys; pairs otherwise
+// and under a position bias.
+int fwd_unit_kind(int B, int H, int H_kv, int N, int window, bool alibi, int sm_count);
 
-// attn_fwd with an optional slope array (NULL: no position bias).  split:
-// 1 / 0 forces split or pair units, -1 lets fwd_split_units decide (callers
-// that cut one problem into several launches pass the whole problem's choice,
-// so that every row is computed as the uncut call computes it).
+// attn_fwd with an optional slope array (NULL: no position bias).  uk: the
+// work-unit kind, or -1 for the test hook's choice, else fwd_unit_kind's
+// (callers that cut one problem into several launches pass the whole
+// problem's kind, so that every row is computed as the uncut call computes it).
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse,
              const float* slopes, int B, int H, int H_kv, int N, int d, int causal, int window,
-             int n_sink, float scale, int dtype, void* stream, int split = -1);
+             int n_sink, float scale, int dtype, void* stream, int uk = -1);
 
 }  // namespace attn_host

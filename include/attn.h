@@ -325,12 +325,16 @@ int attn_test_count_blocks(unsigned long long* counter);
 
 /*
  * attn_test_force_units -- schedule test hook (the paper has no counterpart).
- * attn_fwd runs one of two work-unit shapes, chosen from B, H and N alone:
- * pairs of 128-row query tiles (the two softmax warpgroups take one tile
- * each), or, when pairs would leave SMs idle, single tiles whose key blocks
- * the two warpgroups share out and merge (LSE = log-sum of both halves, O the
- * weighted sum).  Both compute the same function; they may differ in the last
- * bits.  mode 0 forces pairs and 1 single tiles on every later attn_fwd
+ * attn_fwd runs one of three work-unit shapes, chosen from the sizes alone:
+ *   0  pairs of consecutive 128-row query tiles of one head (the two softmax
+ *      warpgroups take one tile each);
+ *   1  single tiles whose key blocks the two warpgroups share out and merge
+ *      (LSE = log-sum of both halves, O the weighted sum), when pairs would
+ *      leave SMs idle;
+ *   2  the same 128 rows of two query heads that share a K/V head (GQA / MQA,
+ *      "USAAIO Lesson 91", slide 32), so each K/V block loaded feeds both.
+ * All compute the same function; 0 and 2 give bitwise-equal results, 1 may
+ * differ in the last bits.  A mode forces that shape on every later attn_fwd
  * launch (ALiBi launches always use pairs); -1 restores the automatic choice
  * (the default).  Process-wide; set it between launches only.  Returns
  * ATTN_OK, or ATTN_ERR_INVALID_ARG for another mode.

@@ -188,9 +188,9 @@ def test_withhold_hook_arguments():
 
 
 def test_force_units_hook_arguments():
-    for bad in (-2, 2, 7):
+    for bad in (-2, 3, 7):
         assert A.test_force_units(bad) == A.ATTN_ERR_INVALID_ARG
-    for mode in (0, 1, -1):
+    for mode in (0, 1, 2, -1):
         assert A.test_force_units(mode) == A.ATTN_OK
 
 

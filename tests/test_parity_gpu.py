@@ -74,13 +74,14 @@ def units():
     A.test_force_units(-1)
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["pairs", "split"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["pairs", "split", "heads"])
 @pytest.mark.parametrize("case", SWEEP, ids=[_id(c) for c in SWEEP])
-def test_sweep_both_unit_shapes(case, mode, units):
-    """Every sweep case with pairs of Q tiles and with single Q tiles whose key
-    blocks the two softmax warpgroups share (the automatic choice takes one of
-    them by problem size): both against the oracle, the 16-bit output the fp32
-    one rounded once."""
+def test_sweep_every_unit_shape(case, mode, units):
+    """Every sweep case with pairs of Q tiles, with single Q tiles whose key
+    blocks the two softmax warpgroups share, and with pairs of query heads
+    that share a K/V head (the automatic choice takes one of them by problem
+    size): each against the oracle, the 16-bit output the fp32 one rounded
+    once."""
     units(mode)
     B, H, Hk, N, d, dt, causal, window, n_sink = case
     q, k, v = random_qkv(B, H, Hk, N, d, dt, seed=N * 131 + d)
@@ -92,6 +93,22 @@ def test_sweep_both_unit_shapes(case, mode, units):
     assert_parity(errors(o16, l16, Or, Lr), round_floor(Or, dt), what="16-bit out")
     assert torch.equal(o16, o32.to(dt)) and torch.equal(l16, l32)
     assert A.get_status() == A.ATTN_OK
+
+
+@pytest.mark.parametrize("case", [(2, 8, 2, 700, 128, BF, 1, 0, 0), (1, 6, 1, 1000, 64, FP, 1, 300, 65),
+                                  (1, 5, 1, 300, 32, BF, 0, 0, 0), (2, 4, 4, 257, 128, BF, 1, 0, 0)])
+def test_head_pair_units_equal_pair_units_bitwise(case, units):
+    """Two query heads of one K/V head per unit compute each row exactly as a
+    pair of Q tiles of one head does (same blocks, same order): the outputs
+    are bitwise equal, odd head counts and G = 1 included."""
+    B, H, Hk, N, d, dt, causal, window, n_sink = case
+    q, k, v = random_qkv(B, H, Hk, N, d, dt, seed=N + H)
+    scale = A.default_scale(d)
+    units(0)
+    o0, l0 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=False)
+    units(2)
+    o2, l2 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=False)
+    assert torch.equal(o0, o2) and torch.equal(l0, l2)
 
 
 @pytest.mark.parametrize("wl", ["c2", "c2c"])

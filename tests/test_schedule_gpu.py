@@ -47,11 +47,11 @@ def test_forward_computes_exactly_the_visited_blocks(case):
     assert got == A.visited_blocks(N, bool(causal), window, n_sink) * B * H
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["pairs", "split"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["pairs", "split", "heads"])
 @pytest.mark.parametrize("case", CASES)
 def test_forward_unit_shapes_compute_exactly_the_visited_blocks(case, mode):
-    """Pairs of Q tiles and single Q tiles shared by both softmax warpgroups
-    compute the same set of score tiles."""
+    """Pairs of Q tiles, single Q tiles shared by both softmax warpgroups and
+    pairs of query heads of one K/V head compute the same set of score tiles."""
     B, H, H_kv, N, d, dt, causal, window, n_sink = case
     q, k, v = (t.cuda() for t in random_qkv(B, H, H_kv, N, d, dt, seed=1))
     assert A.test_force_units(mode) == A.ATTN_OK
