@@ -111,6 +111,34 @@ def test_head_pair_units_equal_pair_units_bitwise(case, units):
     assert torch.equal(o0, o2) and torch.equal(l0, l2)
 
 
+@pytest.mark.parametrize("mode", [1, 2], ids=["split", "heads"])
+@pytest.mark.parametrize("case", [(2, 8, 2, 4096, 128, BF, 1, 0, 0), (1, 12, 3, 4000, 64, FP, 1, 512, 64),
+                                  (4, 8, 1, 1500, 128, BF, 0, 0, 0)])
+def test_unit_kinds_with_several_units_per_cta(case, mode, units):
+    """Split and head-pair units forced on problems with more units than SMs,
+    so that CTAs run several units (warpgroup 1 of a split unit waits for
+    warpgroup 0 to read its half of the previous unit): sampled rows of every
+    head against the oracle, and the whole output against pair units."""
+    B, H, Hk, N, d, dt, causal, window, n_sink = case
+    q, k, v = random_qkv(B, H, Hk, N, d, dt, seed=N + 3 * H)
+    scale = A.default_scale(d)
+    units(mode)
+    o, l = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=True)
+    units(0)
+    o0, l0 = run_gpu(q, k, v, bool(causal), window, n_sink, scale, out_f32=True)
+    rng = np.random.default_rng(5)
+    for b in range(B):
+        for h in range(H):
+            rows = _sample_rows(N, rng, extra=8)
+            Or, Lr = oracle_rows(q, k, v, b, h, rows, bool(causal), window, n_sink, scale)
+            idx = torch.from_numpy(rows)
+            assert_parity(errors(o[b, h, idx], l[b, h, idx], Or, Lr), what=f"head ({b},{h})")
+    if mode == 2:
+        assert torch.equal(o, o0) and torch.equal(l, l0)
+    else:
+        assert (o - o0).abs().max().item() < 1e-2 and (l - l0).abs().max().item() < 1e-5
+
+
 @pytest.mark.parametrize("wl", ["c2", "c2c"])
 def test_small_workloads_split_units_against_oracle_and_pairs(wl, units):
     """c2 / c2c in full run as split units by default; they match the oracle
