@@ -29,7 +29,6 @@ struct DeviceState {
   int* status = nullptr;           // device address of the status word
   uint64_t attr_set = 0;           // one bit per forward kernel instantiation
   uint32_t dec_attr_set = 0;       // one bit per decode kernel instantiation
-  uint32_t dec_small_attr_set = 0; // one bit per small-group decode kernel instantiation
   uint32_t bwd_attr_set = 0;       // one bit per backward kernel instantiation
   // attn_fwd_host: two copy streams and the events that order its chunks,
   // created on its first call on the device and kept (guarded by g_host_mu)
