@@ -853,7 +853,6 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       s_ph ^= 1u;
       tc_fence_after_sync();
       uint32_t sr[128];
-      tmem_ld_32x32b_x128(s_tmem, sr);
       const int c0 = j * BN;
       const bool masked = block_needs_mask(p, r0, c0);
       float m_blk;
@@ -875,7 +874,36 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
       }
       // Logits already scaled (and biased) in sr, instead of raw scores.
       const bool prescaled = (ALIBI && !linear) || (masked && c == 0.f);
-      if (prescaled) {
+      if (!ALIBI && !masked && c >= 0.f) {
+        // Interior block: the raw row maximum of each 32-column chunk is
+        // taken while the next chunk is read from TMEM.
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 32);
+        uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 64);
+        uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 96);
+        float m0 = -INFINITY, m1 = -INFINITY;
+        auto chunk_max = [&](const uint32_t (&x)[32]) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            m0 = max3(m0, __uint_as_float(x[e]), __uint_as_float(x[e + 1]));
+            m1 = max3(m1, __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]));
+          }
+        };
+        tmem_ld_32x32b_x32_start(s_tmem, s0);
+        tmem_wait_ld_x32(s0);
+        tmem_ld_32x32b_x32_start(s_tmem + 32, s1);
+        chunk_max(s0);
+        tmem_wait_ld_x32(s1);
+        tmem_ld_32x32b_x32_start(s_tmem + 64, s2);
+        chunk_max(s1);
+        tmem_wait_ld_x32(s2);
+        tmem_ld_32x32b_x32_start(s_tmem + 96, s3);
+        chunk_max(s2);
+        tmem_wait_ld_x32(s3);
+        chunk_max(s3);
+        m_blk = fmaxf(m0, m1) * c;
+      } else if (prescaled) {
+        tmem_ld_32x32b_x128(s_tmem, sr);
         // Scale first (adding the position bias -slope |i - j|), then drop
         // masked keys with -inf (any sign of scale).  Kept keys of this row,
         // in block-local columns e = j - c0:
@@ -902,6 +930,7 @@ __device__ void softmax_role(const KernelParams& p, const CUtensorMap* tmO, uint
         }
         m_blk = fmaxf(m0, m1);
       } else {
+        tmem_ld_32x32b_x128(s_tmem, sr);
         if (masked) {
           // A masked key gets the raw score -inf (+inf for a negative scale),
           // which the scale turns into -inf; the raw extreme and the exps
