@@ -267,7 +267,7 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = 
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     stream = torch.cuda.current_stream(q.device).cuda_stream
-    with torch.cuda.device(q.device):
+    with _Device(q.device):
         rc = attn_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              lse.data_ptr() if lse is not None else None, ws_ptr, ws_bytes, B, H,
                              H_kv, N_q, N_kv, d, causal, window, n_sink, scale, code, stream)
@@ -340,7 +340,7 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     stream = torch.cuda.current_stream(q.device).cuda_stream
-    with torch.cuda.device(q.device):
+    with _Device(q.device):
         rc = attn_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
                           lse.data_ptr(), alibi_slopes.data_ptr() if alibi_slopes is not None else None,
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws_ptr, ws_bytes, B, H,
@@ -348,6 +348,27 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_bwd")
     return dq, dk, dv
+
+
+class _Device:
+    """Makes `dev` the current CUDA device for a library call; a no-op (no
+    device switch) when it already is, the common case."""
+    __slots__ = ("dev", "ctx")
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.ctx = None
+
+    def __enter__(self):
+        if self.dev.index is not None and self.dev.index != torch.cuda.current_device():
+            self.ctx = torch.cuda.device(self.dev)
+            self.ctx.__enter__()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ctx is not None:
+            self.ctx.__exit__(*exc)
+        return False
 
 
 def _check(q, k, v):
@@ -415,7 +436,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool
         if (alibi_slopes.dtype != torch.float32 or alibi_slopes.device != q.device
                 or tuple(alibi_slopes.shape) != (H,) or not alibi_slopes.is_contiguous()):
             raise ValueError("alibi_slopes must be a contiguous float32 [H] tensor on q's device")
-    with torch.cuda.device(q.device):
+    with _Device(q.device):
         if alibi_slopes is None:
             rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                               lse.data_ptr() if lse is not None else None, B, H, H_kv, N, d,
@@ -465,7 +486,7 @@ def attention_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, st
     code = _dtype_code(q) | (ATTN_OUT_F32 if out_f32 else 0)
     s = (stream or torch.cuda.current_stream(dev)).cuda_stream
     dl = staging.get("lse")
-    with torch.cuda.device(dev):
+    with _Device(dev):
         rc = int(load_library().attn_fwd_host(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
             lse.data_ptr() if lse is not None else None,
