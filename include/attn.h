@@ -94,7 +94,13 @@ enum {
  *   stream cudaStream_t as void*
  *
  * Needs an sm_100 device (B200); other devices give ATTN_ERR_UNSUPPORTED.
- * Returns after the kernel is enqueued.
+ * Returns after the kernel is enqueued.  One launch, with programmatic stream
+ * serialisation: its CTAs may set up (barriers, tensor memory) while the
+ * previous kernel of `stream` drains, and read or write global memory only
+ * after that kernel has completed, so stream order holds.  The kernel allows
+ * the next kernel of `stream` to be scheduled early only if that kernel was
+ * itself launched with programmatic stream serialisation; such a kernel must
+ * wait for it (griddepcontrol.wait) before reading o or lse.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int H_kv, int N, int d, int causal, int window, int n_sink,
@@ -180,7 +186,9 @@ int attn_alibi_slopes(int H, float* slopes);
  * gets one partial (O_s, LSE_s) per range in the workspace, and a second
  * kernel merges them in range order (LSE = ln sum exp(LSE_s),
  * O = sum exp(LSE_s - LSE) O_s), so results are deterministic.  One or two
- * kernel launches on `stream`.
+ * kernel launches on `stream`, both with programmatic stream serialisation as
+ * attn_fwd's (the merge waits for the split kernel before reading the
+ * workspace).
  */
 int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                 void* workspace, long long workspace_bytes, int B, int H, int H_kv, int N_q,
