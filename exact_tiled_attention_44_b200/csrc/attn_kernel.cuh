@@ -154,11 +154,13 @@ __host__ __device__ constexpr uint32_t instr_desc(bool bf16, int m, int n, bool 
 
 // ------------------------------------------------------------ schedule
 
-// One work unit: query rows [q0, q0 + 256) of head (b, h).  Key blocks are
-// iterated as a sink prefix [0, sb) followed by [wlo, hi_max); Q tile t uses
-// block j iff j < sb_t or lo_t <= j < hi_t.  Blocks holding no kept
-// pair for a tile are skipped ("Tiled attention with online softmax": only key
-// blocks at or before the query block; exercise 4: sinks and a window).
+// One work unit of head (b, h): two 128-row Q tiles t = 0, 1 (rows from q0;
+// see decode_unit for the three kinds of unit).  Key blocks are iterated as a
+// sink prefix [0, sb) followed by [wlo, hi_max); in pair and head-pair units
+// Q tile t uses block j iff j < sb_t or lo_t <= j < hi_t.  Blocks holding no
+// kept pair for a tile are skipped ("Tiled attention with online softmax":
+// key blocks past the query block are not visited; exercise 4: sinks and a
+// window).
 struct Unit {
   int bh, b, h, g, q0;
   int n_active;
