@@ -24,7 +24,7 @@ __all__ = [
     "alibi_slopes", "decode", "decode_workspace_bytes", "attn_decode_raw",
     "attn_decode_noalloc_raw", "attention_backward", "attn_bwd_raw", "bwd_workspace_bytes",
     "unmasked_pairs",
-    "visited_blocks", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
+    "visited_blocks", "fwd_unit_kind", "get_status", "set_watchdog_ns", "launch_count", "test_withhold_loads",
     "test_count_blocks", "test_force_units", "error_string",
     "library_path", "load_library", "EXPORTED_SYMBOLS", "ATTN_OK", "ATTN_ERR_INVALID_ARG",
     "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_MISALIGNED", "ATTN_ERR_CUDA", "ATTN_ERR_DEVICE_TIMEOUT",
@@ -44,6 +44,7 @@ ATTN_OUT_F32 = 0x10
 EXPORTED_SYMBOLS = ("attn_fwd", "attn_fwd_host", "attn_fwd_alibi", "attn_alibi_slopes",
                     "attn_decode", "attn_decode_workspace_bytes", "attn_decode_noalloc",
                     "attn_error_string", "attn_unmasked_pairs", "attn_visited_blocks",
+                    "attn_fwd_unit_kind",
                     "attn_get_status", "attn_set_watchdog_ns", "attn_launch_count",
                     "attn_test_withhold_loads", "attn_test_count_blocks", "attn_test_force_units",
                     "attn_bwd", "attn_bwd_workspace_bytes")
@@ -101,6 +102,8 @@ def load_library():
     lib.attn_test_withhold_loads.restype = ci
     lib.attn_test_count_blocks.argtypes = [vp]
     lib.attn_test_count_blocks.restype = ci
+    lib.attn_fwd_unit_kind.argtypes = [ci] * 7
+    lib.attn_fwd_unit_kind.restype = ci
     lib.attn_test_force_units.argtypes = [ci]
     lib.attn_test_force_units.restype = ci
     lib.attn_bwd.argtypes = [vp] * 11 + [ctypes.c_longlong] + [ci] * 8 + [cf, ci, vp]
@@ -123,6 +126,14 @@ def unmasked_pairs(N: int, causal: bool, window: int = 0, n_sink: int = 0) -> in
 def visited_blocks(N: int, causal: bool, window: int = 0, n_sink: int = 0) -> int:
     """128x128 block pairs the kernel's schedule computes for one head."""
     return int(load_library().attn_visited_blocks(N, int(causal), window, n_sink))
+
+
+def fwd_unit_kind(B: int, H: int, H_kv: int, N: int, window: int = 0, alibi: bool = False,
+                  sm_count: int = 0) -> int:
+    """Work-unit shape attn_fwd runs for these sizes (0 tile pairs, 1 split
+    tiles, 2 head pairs; host only, see include/attn.h); sm_count 0 asks the
+    current device."""
+    return int(load_library().attn_fwd_unit_kind(B, H, H_kv, N, window, int(alibi), sm_count))
 
 
 def get_status() -> int:

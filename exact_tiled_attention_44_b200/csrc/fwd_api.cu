@@ -91,6 +91,18 @@ using namespace attn_host;
 
 extern "C" {
 
+int attn_fwd_unit_kind(int B, int H, int H_kv, int N, int window, int alibi, int sm_count) {
+  if (B < 0 || H < 1 || H_kv < 1 || H % H_kv != 0 || N < 0 || window < 0 || sm_count < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (sm_count == 0) {
+    DeviceState* st = nullptr;
+    const int rc = device_state(&st);
+    if (rc != ATTN_OK) return rc;
+    sm_count = st->sm_count;
+  }
+  return fwd_unit_kind(B, H, H_kv, N, window, alibi != 0, sm_count);
+}
+
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int H_kv, int N, int d, int causal, int window, int n_sink, float scale, int dtype,
              void* stream) {

@@ -285,6 +285,23 @@ long long attn_unmasked_pairs(int N, int causal, int window, int n_sink);
 long long attn_visited_blocks(int N, int causal, int window, int n_sink);
 
 /*
+ * attn_fwd_unit_kind -- host only: the work-unit shape attn_fwd (alibi == 0)
+ * or attn_fwd_alibi (alibi != 0) runs for these sizes on a device with
+ * `sm_count` SMs (0: the current device's count, which needs an sm_100
+ * device):
+ *   0  pairs of consecutive 128-row query tiles of one head;
+ *   1  single tiles whose key blocks the two softmax warpgroups share, when
+ *      pairs would leave SMs idle (B * H * ceil(N / 256) < sm_count) and single
+ *      tiles still fit two waves (B * H * ceil(N / 128) <= 2 * sm_count);
+ *   2  the same rows of two query heads sharing a K/V head, for H / H_kv >= 2
+ *      when a row sees at most 4096 keys (min(N, window) <= 4096).
+ * Position-biased launches always use 0.  The result does not depend on
+ * causal, n_sink, d or the data.  Returns ATTN_ERR_INVALID_ARG for B < 0,
+ * H < 1, H_kv < 1, H % H_kv != 0, N < 0, window < 0 or sm_count < 0.
+ */
+int attn_fwd_unit_kind(int B, int H, int H_kv, int N, int window, int alibi, int sm_count);
+
+/*
  * attn_get_status -- reads and clears the device status word of the current
  * device.  Every wait inside the kernel is bounded (about attn_watchdog_ns
  * nanoseconds); a CTA whose wait expires drains its own in-flight copies and

@@ -187,6 +187,49 @@ def test_withhold_hook_arguments():
     assert A.test_withhold_loads(0) == A.ATTN_OK
 
 
+# -------------------------------------------------------- work-unit kind (host only)
+
+@pytest.mark.parametrize("sizes,kind", [
+    ((1, 1, 1, 64, 0, False), 1),          # c1: one tile -> split units
+    ((2, 8, 8, 1024, 0, False), 1),        # c2 / c2c: 64 pairs < 148 SMs, 128 tiles -> split
+    ((4, 16, 16, 4096, 0, False), 0),      # c3: 1024 pairs -> tile pairs
+    ((1, 32, 32, 16384, 0, False), 0),     # c4: MHA -> tile pairs
+    ((8, 32, 1, 8192, 1024, False), 2),    # c5: MQA, rows see 1024 keys -> head pairs
+    ((4, 32, 4, 16384, 0, False), 0),      # GQA with long causal rows -> tile pairs
+    ((4, 32, 8, 4096, 0, False), 2),       # GQA, N = 4096 -> head pairs
+    ((4, 32, 8, 4097, 0, False), 0),       # one key past the head-pair limit
+    ((4, 16, 16, 4096, 0, True), 0),       # a position bias keeps pairs
+    ((2, 8, 8, 1024, 0, True), 0),         # ... even where split units would apply
+    ((1, 148, 148, 256, 0, False), 0),     # 148 pairs: no SM idle -> pairs
+    ((1, 147, 147, 256, 0, False), 1),     # 147 pairs, 294 tiles <= 296 -> split
+    ((1, 100, 100, 384, 0, False), 0),     # 200 pairs >= 148 -> pairs
+    ((1, 60, 60, 640, 0, False), 0),       # 60 heads x 3 pairs = 180 >= 148 -> pairs
+    ((1, 60, 60, 384, 0, False), 1),       # 60 x 2 = 120 pairs, 180 tiles -> split
+])
+def test_unit_kind_rule(sizes, kind):
+    B, H, Hk, N, window, alibi = sizes
+    pairs = B * H * ((N + 255) // 256)
+    tiles = B * H * ((N + 127) // 128)
+    if alibi:
+        expect = 0
+    elif pairs < 148 and tiles <= 296:
+        expect = 1
+    elif H // Hk >= 2 and (window if 0 < window < N else N) <= 4096:
+        expect = 2
+    else:
+        expect = 0
+    got = A.fwd_unit_kind(B, H, Hk, N, window, alibi, 148)
+    assert got == expect == kind
+
+
+def test_unit_kind_arguments():
+    for bad in [(-1, 1, 1, 64, 0, 0, 148), (1, 0, 1, 64, 0, 0, 148), (1, 4, 3, 64, 0, 0, 148),
+                (1, 4, 0, 64, 0, 0, 148), (1, 4, 4, -1, 0, 0, 148), (1, 4, 4, 64, -2, 0, 148),
+                (1, 4, 4, 64, 0, 0, -1)]:
+        assert A.fwd_unit_kind(*bad) == A.ATTN_ERR_INVALID_ARG
+    assert A.fwd_unit_kind(0, 4, 4, 64, 0, False, 148) in (0, 1, 2)   # empty problem: any kind
+
+
 def test_force_units_hook_arguments():
     for bad in (-2, 3, 7):
         assert A.test_force_units(bad) == A.ATTN_ERR_INVALID_ARG
