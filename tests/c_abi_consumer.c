@@ -28,6 +28,10 @@ int main(void) {
   check("unmasked_pairs_full_100", attn_unmasked_pairs(100, 0, 0, 0), 100LL * 100);
   check("visited_blocks_causal_4096", attn_visited_blocks(4096, 1, 0, 0), 32 * 33 / 2);
   check("unmasked_pairs_bad", attn_unmasked_pairs(-1, 1, 0, 0), -1);
+  check("unit_kind_c3", attn_fwd_unit_kind(4, 16, 16, 4096, 0, 0, 148), 0);
+  check("unit_kind_c2", attn_fwd_unit_kind(2, 8, 8, 1024, 0, 0, 148), 1);
+  check("unit_kind_c5", attn_fwd_unit_kind(8, 32, 1, 8192, 1024, 0, 148), 2);
+  check("unit_kind_bad", attn_fwd_unit_kind(1, 4, 3, 64, 0, 0, 148), ATTN_ERR_INVALID_ARG);
 
   /* the pages' ALiBi slopes for H = 8 are 2^-1 .. 2^-8, exact in float */
   float slopes[8];
