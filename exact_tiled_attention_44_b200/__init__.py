@@ -272,9 +272,10 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = 
         out = torch.empty((B, H, N_q, d), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
-    need = decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        need = decode_workspace_bytes(B, H, H_kv, N_q, N_kv, d)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     stream = torch.cuda.current_stream(q.device).cuda_stream
