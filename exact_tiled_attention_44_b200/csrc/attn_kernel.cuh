@@ -16,15 +16,19 @@
 //   warp 8     MMA issue (whole warp, one elected lane issues) + TMEM allocation
 //   warp 9     TMA producer (whole warp, one elected lane issues)
 //   warps 10-11 idle (they hand their registers to the softmax warpgroups)
-// A work unit is (b, h, a pair of adjacent 128-row Q tiles).  Both Q tiles
-// consume the same K/V block stream, so every K/V block loaded from HBM feeds
+// A work unit is, by default, (b, h, a pair of adjacent 128-row Q tiles); for
+// few heads and short sequences one Q tile whose K/V blocks the two softmax
+// warpgroups share out, and for grouped heads with short rows the same 128
+// rows of two query heads of one K/V head (see decode_unit).  Both tiles of a
+// unit consume one K/V block stream, so every K/V block loaded from HBM feeds
 // two 128 x 128 x d MMAs per GEMM.
 //
 // Per K/V block j and Q tile t:
 //   MMA warp   S_t = Q_t K_j^T         (tcgen05.mma, A and B from smem, fp32 in TMEM)
 //   softmax t  reads S_t row-per-thread (tcgen05.ld 32x32b), adds the ALiBi
 //              bias -slope_h |i - j| when asked ("USAAIO Lesson 91", slides
-//              20-23), masks boundary blocks, updates m and l, writes
+//              20-23) folded into the raw scores, masks boundary blocks,
+//              updates m and l, writes
 //              P_t = exp2(s*scale*log2e - m)
 //              as 16-bit over the first half of S_t's columns, and rescales
 //              O_t in TMEM when the max grew by more than 2^8 (lazy rescale:
